@@ -1,0 +1,49 @@
+"""CPU oracle for hybrid Top-k+Top-p block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY. This package is the plain, slow, fp64 statement of
+what the sparse-attention path computes, used to check the CUDA path. Only
+``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its ``cpu_baseline``
+leg and its ``--impl reference`` arm) may import or call it. The product
+package ``block_sparse_attention_row_b200`` never imports it and has no CPU
+fallback; the oracle shares no code with it.
+
+Sources (gist.science summaries; cited by page title and section):
+
+* "SpargeAttention2: Trainable Sparse Attention via Hybrid Top-k+Top-p
+  Masking and Distillation Fine-Tuning" (Hindi and Arabic summaries):
+  §1 Problem Statement (the Top-k and Top-p rules and their failure modes),
+  §2A Hybrid Top-k + Top-p Masking (per-row union), §2C Efficient Kernel
+  Implementation (block-level mask over tiles, masked tiles skipped).
+* "SLA2: Sparse-Linear Attention with Learnable Routing and QAT": §1 Problem
+  Statement and §2B Learnable Router (a compressed score computed from pooled
+  queries and keys).
+* "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
+  Semantic-Aware Permutation": §1 (mean or max pooling of contiguous token
+  blocks) and §2B Centroid-Based Top-p Selection (sort by score, take items
+  until the cumulative score reaches p).
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, hand rows under ``tests/golden/``, invariants, library special
+cases, brute force on tiny inputs). The absolute values of the score matrix
+and of the output on the synthetic workloads have no printed counterpart on
+the pages; beyond those pins they are fixed only by the definitions.
+"""
+from .sparse_attn_oracle import (
+    to_f64,
+    pool_blocks,
+    block_scores,
+    topk_count,
+    topp_threshold,
+    select_row,
+    hybrid_select,
+    hybrid_mask,
+    attend_row,
+    block_sparse_attention,
+    row_sample,
+)
+
+__all__ = [
+    "to_f64", "pool_blocks", "block_scores", "topk_count", "topp_threshold",
+    "select_row", "hybrid_select", "hybrid_mask", "attend_row",
+    "block_sparse_attention", "row_sample",
+]

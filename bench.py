@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark: hybrid Top-k+Top-p block-sparse attention on B200.
+
+One step = the whole path on one layer's worth of synthetic video-DiT
+attention inputs already resident in HBM: the block mask (pool, score,
+select) and then the block-sparse forward over the kept tiles.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config wan]
+  python bench.py --impl reference ...   (the CPU oracle, timed on host cores)
+
+Multi-GPU runs (torchrun, one process per GPU) are weak-scaled replicas: each
+rank runs its own instance of the workload (heads are independent; the path
+has no data exchange). Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse attn ms/call & kept-tile TFLOPS vs bf16 peak; speedup vs own dense"
+UNIT = "TFLOP/s (kept tiles)"
+DEFAULT_CONFIG = "wan"
+FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_fwd_kernel.cuh",
+               "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
+MASK_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
+                "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--k", type=float, default=None)
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--only-step", action="store_true",
+                    help="time only the step loop (used under ncu for the launch list)")
+    return ap.parse_args()
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def profiled_traffic(kind: str, sources) -> dict | None:
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(kind)
+    if not d or d.get("source_hash") != source_hash(sources):
+        return None
+    return d
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the GPU is loaded."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.proc = None
+        self.thread = None
+        self.sel = []
+        try:
+            import torch
+            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
+            self.sel = ["--id=" + str(bus)]
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                self.sel = ["--id=" + vis.split(",")[device_index]]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                clk, mclk, pw = float(r[1]), float(r[2]), float(r[3])
+            except ValueError:
+                continue
+            mx = mclk
+            if pw > 300.0:  # under load
+                sm.append(clk)
+                for n, v in zip(names, r[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:  # short runs: fall back to every sample
+            for r in self.rows:
+                try:
+                    sm.append(float(r[1]))
+                except ValueError:
+                    pass
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------- workload
+def kept_flops(cnt, idx, N, d, bq, bk):
+    """Algorithmic FLOPs of the kept tiles: 4 d x (valid query rows) x (valid keys)."""
+    import torch
+    B, H, n_q = cnt.shape
+    n_k = idx.shape[-1]
+    dev = cnt.device
+    vq = torch.clamp(N - torch.arange(n_q, device=dev) * bq, max=bq).double()
+    vk = torch.clamp(N - torch.arange(n_k, device=dev) * bk, max=bk).double()
+    col = torch.arange(n_k, device=dev)
+    valid = col.view(1, 1, 1, n_k) < cnt.unsqueeze(-1)
+    keys = torch.where(valid, vk[idx.clamp(0, n_k - 1).long()], torch.zeros((), dtype=torch.float64, device=dev))
+    per_row = keys.sum(-1)  # valid keys per row
+    flops = 4.0 * d * (per_row * vq.view(1, 1, n_q)).sum().item()
+    tiles = int(cnt.sum().item())
+    return flops, tiles
+
+
+def dense_flops(B, H, N, d):
+    return 4.0 * B * H * float(N) * float(N) * d
+
+
+def time_events(fn, reps: int, stream) -> list:
+    import torch
+    out = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(a.elapsed_time(b))
+    return out
+
+
+# ----------------------------------------------------------- cpu oracle
+def oracle_sample(cfg, Qh, Kh, Vh, k, p, heads, q_stride, budget_s=None):
+    """Run the CPU oracle on a bounded sample; returns (seconds, kept FLOPs, description)."""
+    import numpy as np
+    import oracle as O
+    t0 = time.perf_counter()
+    flops = 0.0
+    rows_done = 0
+    for h in heads:
+        q = O.to_f64(Qh[0, h])
+        kk = O.to_f64(Kh[0, h])
+        v = O.to_f64(Vh[0, h])
+        P = O.block_scores(O.pool_blocks(q, cfg.bq), O.pool_blocks(kk, cfg.bk), cfg.d)
+        cnt, idx, _ = O.hybrid_select(P.astype(np.float32), k, p)
+        for i in range(0, cfg.n_q, q_stride):
+            lo, hi = i * cfg.bq, min(cfg.N, (i + 1) * cfg.bq)
+            kept = idx[i, :cnt[i]]
+            O.attend_row(q[lo:hi], kk, v, kept, cfg.bk)
+            nkeys = sum(min(cfg.bk, cfg.N - j * cfg.bk) for j in kept)
+            flops += 4.0 * cfg.d * (hi - lo) * nkeys
+            rows_done += 1
+            if budget_s is not None and time.perf_counter() - t0 > budget_s:
+                break
+    dt = time.perf_counter() - t0
+    desc = (f"{cfg.name}: heads {list(heads)} (mask of the whole head, then attention for every "
+            f"{q_stride}th query block: {rows_done} rows), fp64 numpy")
+    return dt, flops, desc
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def host_copies(cfg, rank):
+    from synth import make_qkv_custom
+    return make_qkv_custom(cfg.B, cfg.H, cfg.N, cfg.d, seed=cfg.seed + 100 * rank, device="cuda",
+                           grid=cfg.grid, positional_field=cfg.positional_field,
+                           sink_heads=cfg.sink_heads, uniform_heads=cfg.uniform_heads, bk_sink=cfg.bk)
+
+
+# ------------------------------------------------------------ reference
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from synth import CONFIGS, make_qkv
+    cfg = CONFIGS[args.config]
+    k = args.k if args.k is not None else cfg.k
+    p = args.p if args.p is not None else cfg.p
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    Q, K, V = make_qkv(cfg, device=dev)
+    Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+    del Q, K, V
+    heads_all = list(range(cfg.H))
+    q_stride = max(1, cfg.n_q // 4)
+    times, flops = [], []
+    desc = ""
+    for s in range(args.warmup + args.steps):
+        h = heads_all[s % cfg.H]
+        dt, fl, desc = oracle_sample(cfg, Qh, Kh, Vh, k, p, [h], q_stride)
+        if s >= args.warmup:
+            times.append(dt)
+            flops.append(fl)
+    value = sum(flops) / sum(times) / 1e12
+    ms = 1e3 * sum(times) / len(times)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
+                       "bq": cfg.bq, "bk": cfg.bk, "k": k, "p": p},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": "per step one head (cycling): " + desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    from block_sparse_attention_row_b200 import (check_device_error, mask_workspace_bytes,
+                                                 sparse_attn_fwd, sparse_attn_fwd_dense,
+                                                 sparse_attn_mask, load_library)
+    from synth import CONFIGS
+    load_library()
+    cfg = CONFIGS[args.config]
+    k = args.k if args.k is not None else cfg.k
+    p = args.p if args.p is not None else cfg.p
+    B, H, N, d, bq, bk = cfg.B, cfg.H, cfg.N, cfg.d, cfg.bq, cfg.bk
+    n_q, n_k = cfg.n_q, cfg.n_k
+    Q, K, V = host_copies(cfg, rank)
+    stream = torch.cuda.current_stream(dev)
+    out = {"cnt": torch.empty((B, H, n_q), dtype=torch.int32, device=dev),
+           "idx": torch.empty((B, H, n_q, n_k), dtype=torch.int32, device=dev)}
+    ws = torch.empty(mask_workspace_bytes(B, H, N, d, bq, bk), dtype=torch.uint8, device=dev)
+    O = torch.empty_like(Q)
+
+    def do_mask():
+        sparse_attn_mask(Q, K, bq, bk, k, p, out=out, workspace=ws)
+
+    def do_fwd():
+        sparse_attn_fwd(Q, K, V, out["cnt"], out["idx"], bq, bk, out=O)
+
+    def step():
+        do_mask()
+        do_fwd()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    check_device_error(dev)
+    fl, tiles = kept_flops(out["cnt"], out["idx"], N, d, bq, bk)
+    sparsity = 1.0 - tiles / float(B * H * n_q * n_k)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_step = e0.elapsed_time(e1) / max(args.steps, 1)
+    if world > 1:
+        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+        f = torch.tensor([fl], device=dev, dtype=torch.float64)
+        dist.all_reduce(f, op=dist.ReduceOp.SUM)
+        total_flops = float(f.item())
+    else:
+        total_flops = fl
+    value = total_flops / (ms_step * 1e-3) / 1e12
+
+    extra = {}
+    if not args.only_step:
+        reps = 10
+        mask_ms = statistics.median(time_events(do_mask, reps, stream))
+        fwd_ms = statistics.median(time_events(do_fwd, reps, stream))
+        dense_ms = None
+        if not args.no_dense:
+            def do_dense():
+                sparse_attn_fwd_dense(Q, K, V, bq, bk, out=O)
+            dense_ms = statistics.median(time_events(do_dense, 3, stream))
+        check_device_error(dev)
+        # end to end through the public API with host buffers (pinned)
+        Qh = Q.cpu().pin_memory()
+        Kh = K.cpu().pin_memory()
+        Vh = V.cpu().pin_memory()
+        Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        Qd, Kd, Vd = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+        def e2e_step():
+            Qd.copy_(Qh, non_blocking=True)
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            sparse_attn_mask(Qd, Kd, bq, bk, k, p, out=out, workspace=ws)
+            sparse_attn_fwd(Qd, Kd, Vd, out["cnt"], out["idx"], bq, bk, out=O)
+            Oh.copy_(O, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_reps = max(3, min(args.steps, 20))
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_reps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / e2e_reps
+        check_device_error(dev)
+        peaks = measured_peaks()
+        fwd_tflops = fl / (fwd_ms * 1e-3) / 1e12
+        mask_bytes = 2.0 * B * H * N * d * 2 + 4.0 * (tiles + B * H * n_q)
+        mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
+        tr = profiled_traffic("fwd", FWD_SOURCES)
+        extra = {
+            "ms_per_call": {"mask": mask_ms, "fwd": fwd_ms, "mask_plus_fwd": mask_ms + fwd_ms,
+                            "dense_fwd": dense_ms},
+            "block_sparsity": sparsity,
+            "kept_tiles": tiles,
+            "kept_tile_tflops": {"fwd": fwd_tflops, "step": fl / (ms_step * 1e-3) / 1e12},
+            "speedup_vs_own_dense": None if dense_ms is None else {
+                "fwd_only": dense_ms / fwd_ms, "mask_plus_fwd": dense_ms / (mask_ms + fwd_ms),
+                "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - sparsity)},
+            "dense_tflops": None if dense_ms is None else dense_flops(B, H, N, d) / (dense_ms * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
+                         "traffic": None if tr is None else tr["bytes_per_launch"],
+                         "kernel": "sparse_fwd_kernel", "peak_source": peaks["source"] + " (burst)",
+                         "frac_of_sustained": None if not peaks.get("bf16_tflops_sustained") else
+                         fwd_tflops / peaks["bf16_tflops_sustained"]},
+            "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": peaks["hbm_gbs"],
+                              "unit": "GB/s", "frac": mask_gbs / peaks["hbm_gbs"],
+                              "algorithmic_bytes": mask_bytes,
+                              "kernels": "pool_kernel + score_kernel + select_kernel"},
+            "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
+        }
+    clk = clocks.stop()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only_step:
+        Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
+        heads = sorted({min(H - 1, h) for h in (0, 5, 10, 15, 25, 35)})
+        dt, cfl, desc = oracle_sample(cfg, Qh, Kh, Vh, k, p, heads, max(1, n_q // 64), budget_s=30.0)
+        extra["cpu_baseline"] = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": cpu_threads(),
+                                 "kind": "oracle", "sample": desc, "seconds": dt}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": cfg.name, "B": B, "H": H, "N": N, "d": d, "bq": bq, "bk": bk,
+                           "k": k, "p": p, "parallelism": f"replicas x{world} (weak)",
+                           "l2": "inputs larger than L2 (Q,K,V %.0f MB vs 126 MB); no flush" %
+                                 (3 * Q.numel() * 2 / 1e6)},
+                "gpu_launches": 4 * args.steps,
+                "clocks": clk}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,235 @@
+"""Python binding of libsparse_attn.so (the C ABI in include/sparse_attn.h).
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no CPU path: inputs must be CUDA tensors and the built library must
+be present, otherwise these functions raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional
+
+import torch
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libsparse_attn.so")
+
+SA_OK = 0
+STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_CUDA",
+                4: "SA_ERR_TIMEOUT", 5: "SA_ERR_DEVICE_ASSERT"}
+
+# Every entry point declared in include/sparse_attn.h.
+EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_select",
+            "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_check_device_error",
+            "sparse_attn_last_error", "sparse_attn_version")
+
+
+class SaShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("bq", ctypes.c_int32), ("bk", ctypes.c_int32)]
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, func: str, status: int, message: str):
+        self.status = status
+        super().__init__(f"{func}: {STATUS_NAMES.get(status, status)}: {message}")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libsparse_attn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "block_sparse_attention_row_b200.build.build()")
+        lib = ctypes.CDLL(path)
+        vp, i32p, u8p, f32p = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+        sp = ctypes.POINTER(SaShape)
+        lib.sparse_attn_mask_workspace_bytes.argtypes = [sp]
+        lib.sparse_attn_mask_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_mask.argtypes = [sp, vp, vp, ctypes.c_double, ctypes.c_double, i32p, i32p,
+                                         u8p, f32p, vp, vp]
+        lib.sparse_attn_mask.restype = ctypes.c_int
+        lib.sparse_attn_select.argtypes = [sp, f32p, ctypes.c_double, ctypes.c_double, i32p, i32p,
+                                           u8p, vp]
+        lib.sparse_attn_select.restype = ctypes.c_int
+        lib.sparse_attn_fwd.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, f32p, vp]
+        lib.sparse_attn_fwd.restype = ctypes.c_int
+        lib.sparse_attn_fwd_dense.argtypes = [sp, vp, vp, vp, vp, f32p, vp]
+        lib.sparse_attn_fwd_dense.restype = ctypes.c_int
+        lib.sparse_attn_check_device_error.argtypes = [vp]
+        lib.sparse_attn_check_device_error.restype = ctypes.c_int
+        lib.sparse_attn_last_error.argtypes = []
+        lib.sparse_attn_last_error.restype = ctypes.c_char_p
+        lib.sparse_attn_version.argtypes = []
+        lib.sparse_attn_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def _check(func: str, status: int) -> None:
+    if status != SA_OK:
+        msg = load_library().sparse_attn_last_error().decode(errors="replace")
+        raise SparseAttnError(func, status, msg)
+
+
+def make_shape(B: int, H: int, N: int, d: int, bq: int, bk: int) -> SaShape:
+    return SaShape(int(B), int(H), int(N), int(d), int(bq), int(bk))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_qkv(*ts: torch.Tensor) -> None:
+    ref = ts[0]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("sparse attention runs on CUDA tensors only (no CPU path)")
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("Q, K, V must be contiguous bf16 tensors of shape [B, H, N, d]")
+        if t.shape != ref.shape or t.device != ref.device:
+            raise ValueError("Q, K, V must share shape and device")
+
+
+def num_blocks(N: int, bq: int, bk: int):
+    return -(-N // bq), -(-N // bk)
+
+
+def mask_workspace_bytes(B, H, N, d, bq, bk) -> int:
+    shape = make_shape(B, H, N, d, bq, bk)
+    return int(load_library().sparse_attn_mask_workspace_bytes(ctypes.byref(shape)))
+
+
+def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: float, p: float, *,
+                     want_mask: bool = False, want_P: bool = False, out: Optional[dict] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Block mask of hybrid Top-k+Top-p selection: {'cnt', 'idx'[, 'mask', 'P']}.
+
+    cnt int32 [B,H,n_q]; idx int32 [B,H,n_q,n_k] (first cnt entries valid,
+    ascending); mask uint8 [B,H,n_q,n_k]; P fp32 [B,H,n_q,n_k]. Pass `out`
+    (a dict holding those tensors) and `workspace` to avoid allocations.
+    """
+    _check_qkv(Q, K)
+    lib = load_library()
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = Q.device
+    shape = make_shape(B, H, N, d, bq, bk)
+    res = dict(out) if out is not None else {}
+    if "cnt" not in res:
+        res["cnt"] = torch.empty((B, H, n_q), dtype=torch.int32, device=dev)
+    if "idx" not in res:
+        res["idx"] = torch.empty((B, H, n_q, n_k), dtype=torch.int32, device=dev)
+    if want_mask and "mask" not in res:
+        res["mask"] = torch.empty((B, H, n_q, n_k), dtype=torch.uint8, device=dev)
+    if want_P and "P" not in res:
+        res["P"] = torch.empty((B, H, n_q, n_k), dtype=torch.float32, device=dev)
+    if workspace is None:
+        nbytes = int(lib.sparse_attn_mask_workspace_bytes(ctypes.byref(shape)))
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    st = lib.sparse_attn_mask(ctypes.byref(shape), _ptr(Q), _ptr(K), float(k), float(p),
+                              _ptr(res["cnt"]), _ptr(res["idx"]), _ptr(res.get("mask")),
+                              _ptr(res.get("P")), _ptr(workspace), _stream(dev, stream))
+    _check("sparse_attn_mask", st)
+    return res
+
+
+def sparse_attn_select(P: torch.Tensor, N: int, d: int, bq: int, bk: int, k: float, p: float, *,
+                       want_mask: bool = False, stream=None) -> dict:
+    """Selection alone on a given fp32 score matrix P [B,H,n_q,n_k]."""
+    if not P.is_cuda or P.dtype != torch.float32 or not P.is_contiguous() or P.dim() != 4:
+        raise ValueError("P must be a contiguous fp32 CUDA tensor [B, H, n_q, n_k]")
+    lib = load_library()
+    B, H, n_q, n_k = P.shape
+    if (n_q, n_k) != num_blocks(N, bq, bk):
+        raise ValueError("P's block counts do not match N, bq, bk")
+    shape = make_shape(B, H, N, d, bq, bk)
+    dev = P.device
+    res = {"cnt": torch.empty((B, H, n_q), dtype=torch.int32, device=dev),
+           "idx": torch.empty((B, H, n_q, n_k), dtype=torch.int32, device=dev)}
+    if want_mask:
+        res["mask"] = torch.empty((B, H, n_q, n_k), dtype=torch.uint8, device=dev)
+    st = lib.sparse_attn_select(ctypes.byref(shape), _ptr(P), float(k), float(p), _ptr(res["cnt"]),
+                                _ptr(res["idx"]), _ptr(res.get("mask")), _stream(dev, stream))
+    _check("sparse_attn_select", st)
+    return res
+
+
+def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cnt: torch.Tensor,
+                    idx: torch.Tensor, bq: int, bk: int, *, want_lse: bool = False,
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                    stream=None):
+    """Block-sparse attention over the kept blocks: O bf16 [B,H,N,d] (, lse fp32 [B,H,N])."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    for t, shp in ((cnt, (B, H, n_q)), (idx, (B, H, n_q, n_k))):
+        if t.dtype != torch.int32 or not t.is_contiguous() or tuple(t.shape) != shp or t.device != Q.device:
+            raise ValueError(f"index tensor must be contiguous int32 {shp} on {Q.device}")
+    lib = load_library()
+    shape = make_shape(B, H, N, d, bq, bk)
+    O = out if out is not None else torch.empty_like(Q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    st = lib.sparse_attn_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(cnt), _ptr(idx),
+                             _ptr(O), _ptr(lse), _stream(Q.device, stream))
+    _check("sparse_attn_fwd", st)
+    return (O, lse) if want_lse else O
+
+
+def sparse_attn_fwd_dense(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bq: int, bk: int, *,
+                          want_lse: bool = False, out: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None, stream=None):
+    """Same kernel with every key block kept (full attention)."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    lib = load_library()
+    shape = make_shape(B, H, N, d, bq, bk)
+    O = out if out is not None else torch.empty_like(Q)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    st = lib.sparse_attn_fwd_dense(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                   _ptr(lse), _stream(Q.device, stream))
+    _check("sparse_attn_fwd_dense", st)
+    return (O, lse) if want_lse else O
+
+
+def sparse_attn(Q, K, V, bq: int, bk: int, k: float, p: float, *, stream=None):
+    """The whole path: mask then block-sparse forward. Returns (O, cnt, idx)."""
+    m = sparse_attn_mask(Q, K, bq, bk, k, p, stream=stream)
+    O = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, bk, stream=stream)
+    return O, m["cnt"], m["idx"]
+
+
+def check_device_error(device=None, stream=None) -> None:
+    """Synchronise and raise if a kernel recorded an error since the last check."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    st = load_library().sparse_attn_check_device_error(_stream(dev, stream))
+    _check("sparse_attn_check_device_error", st)
+
+
+def topk_count(k: float, n_k: int) -> int:
+    """Host copy of the library's Top-k count rule, for reporting only."""
+    if k >= 1.0:
+        return n_k
+    return min(n_k, max(0, math.ceil(k * n_k - 1e-9)))
+
+
+def version() -> str:
+    return load_library().sparse_attn_version().decode()

@@ -1,0 +1,136 @@
+/*
+ * sparse_attn.h - C ABI of the hybrid Top-k+Top-p block-sparse attention
+ * library (libsparse_attn.so), written for NVIDIA B200 (sm_100a).
+ *
+ * The method is the one summarised in "SpargeAttention2: Trainable Sparse
+ * Attention via Hybrid Top-k+Top-p Masking and Distillation Fine-Tuning"
+ * (gist.science summaries, Hindi and Arabic):
+ *   §1 Problem Statement   - the Top-k rule (keep the top k of a row) and the
+ *                            Top-p rule (keep entries until their cumulative
+ *                            probability reaches p), and where each fails;
+ *   §2A Hybrid Masking     - per row, keep the union of both selections;
+ *   §2C Kernel             - a FlashAttention-style kernel applies that mask
+ *                            per tile and skips the matmul and softmax of
+ *                            masked tiles.
+ * The block scores come from mean-pooled queries and keys, as in "SLA2:
+ * Sparse-Linear Attention with Learnable Routing and QAT" §1 and §2B (a
+ * compressed score from pooled Q and K) and "Sparse VideoGen2" §1 (mean
+ * pooling of contiguous token blocks).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are dense, row-major, with no padding:
+ *     Q, K, V, O   bf16  [B, H, N, d]     (token-major within a head)
+ *     cnt          int32 [B, H, n_q]
+ *     idx          int32 [B, H, n_q, n_k] (row capacity n_k)
+ *     mask         uint8 [B, H, n_q, n_k]
+ *     P            fp32  [B, H, n_q, n_k]
+ *     lse          fp32  [B, H, N]        (natural log)
+ *   where n_q = ceil(N / bq) and n_k = ceil(N / bk).
+ * - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *   caller allocates and owns every buffer. The library allocates no memory
+ *   per call; it keeps one small device error record per loaded module.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream). Calls only enqueue work; results are ready when the stream is.
+ * - Supported shapes: d in {64, 128}; bq in {64, 128}; bk = 64;
+ *   1 <= N, n_k <= 8192; B*H <= 65535. Pointers must be 16-byte aligned.
+ * - Return value: SA_OK, or an error code with a message readable through
+ *   sparse_attn_last_error() (thread-local). Argument errors are detected on
+ *   the host before anything is enqueued. Errors raised inside a kernel
+ *   (a bounded wait that ran out, an index out of range) are recorded on the
+ *   device and reported by sparse_attn_check_device_error().
+ * - Inputs must be finite; NaN or Inf propagation is unspecified.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, k/p out of range, misaligned */
+    SA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
+    SA_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed */
+    SA_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (device side) */
+    SA_ERR_DEVICE_ASSERT = 5  /* a kernel found an invalid index list (device side) */
+} sa_status;
+
+typedef struct {
+    int32_t B, H, N, d, bq, bk;
+} sa_shape;
+
+/* Bytes of device workspace sparse_attn_mask needs for `shape` (pooled Q and
+ * K, and the fp32 block-logit matrix). 0 on an invalid shape. */
+size_t sparse_attn_mask_workspace_bytes(const sa_shape* shape);
+
+/* Steps 1-3 of the path: block mask from Q and K.
+ *   1. Qbar_i / Kbar_j = mean of the valid tokens of query block i (bq
+ *      tokens) and key block j (bk tokens);
+ *   2. P = row softmax of Qbar Kbar^T / sqrt(d), fp32;
+ *   3. per row, keep the union of the Top-k set (the ceil(k * n_k) highest
+ *      scores; k >= 1 keeps all) and the Top-p set (the shortest prefix of
+ *      the score order whose mass reaches p of the row total; p >= 1 keeps
+ *      all). The score order is by P descending, equal scores by lower
+ *      index; mass is counted in 31-bit fixed point, floor(P * 2^31), and
+ *      the target is ceil(p * W) in double, W the row's fixed-point total.
+ *      The selection is exact given P: any order of the reductions gives the
+ *      same kept set.
+ * Inputs:  Q, K bf16 [B,H,N,d]; k, p in [0, 1], not both 0.
+ * Outputs: cnt[b,h,i] = number of kept key blocks; idx[b,h,i,0:cnt] = kept
+ *          key-block indices, ascending (entries past cnt are not written);
+ *          mask (optional, may be NULL) = 1 for kept blocks, 0 otherwise;
+ *          P_out (optional, may be NULL) = the fp32 scores the selection
+ *          used.
+ * workspace: device buffer of sparse_attn_mask_workspace_bytes(shape) bytes,
+ *          256-byte aligned; its contents are scratch. */
+sa_status sparse_attn_mask(const sa_shape* shape, const void* Q, const void* K,
+                           double k, double p,
+                           int32_t* cnt, int32_t* idx,
+                           uint8_t* mask_or_null, float* P_out_or_null,
+                           void* workspace, void* stream);
+
+/* Step 3 alone, on a caller-supplied fp32 score matrix P [B,H,n_q,n_k]
+ * (rows of non-negative finite values). Same selection code and outputs as
+ * sparse_attn_mask; used to check the selection bit for bit. */
+sa_status sparse_attn_select(const sa_shape* shape, const float* P, double k, double p,
+                             int32_t* cnt, int32_t* idx, uint8_t* mask_or_null,
+                             void* stream);
+
+/* Step 4: block-sparse attention over the kept tiles only (SpargeAttention2
+ * §2C). For every query block i of every (b, h):
+ *   O[rows of i] = softmax(Q_i K_u^T / sqrt(d)) V_u over the tokens u of the
+ *   key blocks idx[b,h,i,0:cnt[b,h,i]] (tokens >= N excluded);
+ * no work is issued for key blocks not in the list. A row with cnt = 0 gets
+ * O = 0 and lse = -inf. Index entries must lie in [0, n_k); an entry outside
+ * is skipped and reported as SA_ERR_DEVICE_ASSERT.
+ * Inputs: Q, K, V bf16 [B,H,N,d]; cnt, idx as produced by sparse_attn_mask.
+ * Outputs: O bf16 [B,H,N,d]; lse (optional) fp32 [B,H,N]. */
+sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                          const int32_t* cnt, const int32_t* idx,
+                          void* O, float* lse_or_null, void* stream);
+
+/* Step 4 with every key block kept (full attention through the same kernel;
+ * no index list is read). The reference point for the sparse speed-up. */
+sa_status sparse_attn_fwd_dense(const sa_shape* shape, const void* Q, const void* K,
+                                const void* V, void* O, float* lse_or_null, void* stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded since
+ * the last call (SA_OK if none) and clears the record. */
+sa_status sparse_attn_check_device_error(void* stream);
+
+/* Message of the last error returned on this host thread ("" if none). */
+const char* sparse_attn_last_error(void);
+
+/* Library version string. */
+const char* sparse_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse attn ms/call & kept-tile TFLOPS vs bf16 peak; speedup vs own dense"
 UNIT = "TFLOP/s (kept tiles)"
 DEFAULT_CONFIG = "wan"
-FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_fwd_kernel.cuh",
+FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_fwd2_kernel.cuh",
                "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
 MASK_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
                 "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
@@ -99,12 +99,10 @@ class ClockSampler:
         self.sel = []
         try:
             import torch
-            bus = torch.cuda.get_device_properties(device_index).pci_bus_id
-            self.sel = ["--id=" + str(bus)]
+            pr = torch.cuda.get_device_properties(device_index)
+            self.sel = ["--id=%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)]
         except Exception:
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-            if vis:
-                self.sel = ["--id=" + vis.split(",")[device_index]]
+            self.sel = []
 
     def start(self):
         try:
@@ -174,6 +172,26 @@ def kept_flops(cnt, idx, N, d, bq, bk):
     return flops, tiles
 
 
+def aggregate_over_ranks(ms_step: float, flops: float, world: int, device):
+    """Whole-job figures of a weak-scaled run: the slowest rank's step time and
+    the kept-tile FLOPs summed over ranks (every rank takes the same two
+    collective steps in the same order)."""
+    if world <= 1:
+        return ms_step, flops
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms_step], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    f = torch.tensor([flops], device=device, dtype=torch.float64)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each weak-scaled replica draws its own instance of the workload."""
+    return base_seed + 100 * rank
+
+
 def dense_flops(B, H, N, d):
     return 4.0 * B * H * float(N) * float(N) * d
 
@@ -234,7 +252,7 @@ def cpu_threads() -> int:
 
 def host_copies(cfg, rank):
     from synth import make_qkv_custom
-    return make_qkv_custom(cfg.B, cfg.H, cfg.N, cfg.d, seed=cfg.seed + 100 * rank, device="cuda",
+    return make_qkv_custom(cfg.B, cfg.H, cfg.N, cfg.d, seed=rank_seed(cfg.seed, rank), device="cuda",
                            grid=cfg.grid, positional_field=cfg.positional_field,
                            sink_heads=cfg.sink_heads, uniform_heads=cfg.uniform_heads, bk_sink=cfg.bk)
 
@@ -345,15 +363,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     ms_step = e0.elapsed_time(e1) / max(args.steps, 1)
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-        f = torch.tensor([fl], device=dev, dtype=torch.float64)
-        dist.all_reduce(f, op=dist.ReduceOp.SUM)
-        total_flops = float(f.item())
-    else:
-        total_flops = fl
+    ms_step, total_flops = aggregate_over_ranks(ms_step, fl, world, dev)
     value = total_flops / (ms_step * 1e-3) / 1e12
 
     extra = {}
@@ -367,6 +377,23 @@ def run_ours(args):
                 sparse_attn_fwd_dense(Q, K, V, bq, bk, out=O)
             dense_ms = statistics.median(time_events(do_dense, 3, stream))
         check_device_error(dev)
+        # The ~95%-sparsity operating point: Top-k alone at the same k (p = 0)
+        # on the same inputs, where the attention does 1/20 of the dense work.
+        out95 = {"cnt": torch.empty_like(out["cnt"]), "idx": torch.empty_like(out["idx"])}
+        O95 = torch.empty_like(O)
+
+        def do_mask95():
+            sparse_attn_mask(Q, K, bq, bk, k, 0.0, out=out95, workspace=ws)
+
+        def do_fwd95():
+            sparse_attn_fwd(Q, K, V, out95["cnt"], out95["idx"], bq, bk, out=O95)
+
+        do_mask95()
+        fl95, tiles95 = kept_flops(out95["cnt"], out95["idx"], N, d, bq, bk)
+        mask95_ms = statistics.median(time_events(do_mask95, reps, stream))
+        fwd95_ms = statistics.median(time_events(do_fwd95, reps, stream))
+        check_device_error(dev)
+        s95 = 1.0 - tiles95 / float(B * H * n_q * n_k)
         # end to end through the public API with host buffers (pinned)
         Qh = Q.cpu().pin_memory()
         Kh = K.cpu().pin_memory()
@@ -410,10 +437,18 @@ def run_ours(args):
                 "fwd_only": dense_ms / fwd_ms, "mask_plus_fwd": dense_ms / (mask_ms + fwd_ms),
                 "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - sparsity)},
             "dense_tflops": None if dense_ms is None else dense_flops(B, H, N, d) / (dense_ms * 1e-3) / 1e12,
+            "sparsity_95_point": {
+                "k": k, "p": 0.0, "block_sparsity": s95, "kept_tiles": tiles95,
+                "ms_per_call": {"mask": mask95_ms, "fwd": fwd95_ms},
+                "kept_tile_tflops_fwd": fl95 / (fwd95_ms * 1e-3) / 1e12,
+                "frac_of_bf16_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / measured_peaks()["bf16_tflops"],
+                "speedup_vs_own_dense": None if dense_ms is None else {
+                    "fwd_only": dense_ms / fwd95_ms, "mask_plus_fwd": dense_ms / (mask95_ms + fwd95_ms),
+                    "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - s95)}},
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
                          "traffic": None if tr is None else tr["bytes_per_launch"],
-                         "kernel": "sparse_fwd_kernel", "peak_source": peaks["source"] + " (burst)",
+                         "kernel": "sparse_fwd2_kernel", "peak_source": peaks["source"] + " (burst)",
                          "frac_of_sustained": None if not peaks.get("bf16_tflops_sustained") else
                          fwd_tflops / peaks["bf16_tflops_sustained"]},
             "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": peaks["hbm_gbs"],

@@ -13,7 +13,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libsparse_attn.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["sa_lib.cu"]
-DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_fwd_kernel.cuh", "sa_status_codes.h"]
+DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_fwd2_kernel.cuh",
+        "sa_status_codes.h"]
 
 
 def nvcc_path() -> str:

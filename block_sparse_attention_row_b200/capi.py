@@ -19,13 +19,14 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libsparse_attn.so")
 
 SA_OK = 0
+SA_BF16, SA_F32 = 0, 1
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_CUDA",
                 4: "SA_ERR_TIMEOUT", 5: "SA_ERR_DEVICE_ASSERT"}
 
-# Every entry point declared in include/sparse_attn.h.
+# Every entry point declared in include/sparse_attn.h and include/sparse_attn_testing.h.
 EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_select",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_check_device_error",
-            "sparse_attn_last_error", "sparse_attn_version")
+            "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_exp2_poly")
 
 
 class SaShape(ctypes.Structure):
@@ -63,14 +64,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_select.argtypes = [sp, f32p, ctypes.c_double, ctypes.c_double, i32p, i32p,
                                            u8p, vp]
         lib.sparse_attn_select.restype = ctypes.c_int
-        lib.sparse_attn_fwd.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, f32p, vp]
+        lib.sparse_attn_fwd.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, ctypes.c_int, f32p, vp]
         lib.sparse_attn_fwd.restype = ctypes.c_int
-        lib.sparse_attn_fwd_dense.argtypes = [sp, vp, vp, vp, vp, f32p, vp]
+        lib.sparse_attn_fwd_dense.argtypes = [sp, vp, vp, vp, vp, ctypes.c_int, f32p, vp]
         lib.sparse_attn_fwd_dense.restype = ctypes.c_int
         lib.sparse_attn_check_device_error.argtypes = [vp]
         lib.sparse_attn_check_device_error.restype = ctypes.c_int
         lib.sparse_attn_last_error.argtypes = []
         lib.sparse_attn_last_error.restype = ctypes.c_char_p
+        lib.sparse_attn_test_exp2_poly.argtypes = [vp, vp, ctypes.c_int64, vp]
+        lib.sparse_attn_test_exp2_poly.restype = ctypes.c_int
         lib.sparse_attn_version.argtypes = []
         lib.sparse_attn_version.restype = ctypes.c_char_p
         _lib = lib
@@ -171,11 +174,24 @@ def sparse_attn_select(P: torch.Tensor, N: int, d: int, bq: int, bk: int, k: flo
     return res
 
 
+def _out_tensor(Q: torch.Tensor, out: Optional[torch.Tensor], out_dtype: torch.dtype):
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    if out is None:
+        return torch.empty(Q.shape, dtype=out_dtype, device=Q.device)
+    if out.dtype != out_dtype or out.shape != Q.shape or not out.is_contiguous() or out.device != Q.device:
+        raise ValueError("out must be a contiguous tensor of Q's shape and out_dtype")
+    return out
+
+
 def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cnt: torch.Tensor,
                     idx: torch.Tensor, bq: int, bk: int, *, want_lse: bool = False,
                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                    stream=None):
-    """Block-sparse attention over the kept blocks: O bf16 [B,H,N,d] (, lse fp32 [B,H,N])."""
+                    out_dtype: torch.dtype = torch.bfloat16, stream=None):
+    """Block-sparse attention over the kept blocks: O [B,H,N,d] (, lse fp32 [B,H,N]).
+
+    O is bf16 by default; out_dtype=torch.float32 returns the kernel's fp32
+    result, of which the bf16 output is the round-to-nearest-even."""
     _check_qkv(Q, K, V)
     B, H, N, d = Q.shape
     n_q, n_k = num_blocks(N, bq, bk)
@@ -184,28 +200,31 @@ def sparse_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cnt: torc
             raise ValueError(f"index tensor must be contiguous int32 {shp} on {Q.device}")
     lib = load_library()
     shape = make_shape(B, H, N, d, bq, bk)
-    O = out if out is not None else torch.empty_like(Q)
+    O = _out_tensor(Q, out, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     st = lib.sparse_attn_fwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(cnt), _ptr(idx),
-                             _ptr(O), _ptr(lse), _stream(Q.device, stream))
+                             _ptr(O), SA_F32 if O.dtype == torch.float32 else SA_BF16, _ptr(lse),
+                             _stream(Q.device, stream))
     _check("sparse_attn_fwd", st)
     return (O, lse) if want_lse else O
 
 
 def sparse_attn_fwd_dense(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bq: int, bk: int, *,
                           want_lse: bool = False, out: Optional[torch.Tensor] = None,
-                          lse: Optional[torch.Tensor] = None, stream=None):
+                          lse: Optional[torch.Tensor] = None,
+                          out_dtype: torch.dtype = torch.bfloat16, stream=None):
     """Same kernel with every key block kept (full attention)."""
     _check_qkv(Q, K, V)
     B, H, N, d = Q.shape
     lib = load_library()
     shape = make_shape(B, H, N, d, bq, bk)
-    O = out if out is not None else torch.empty_like(Q)
+    O = _out_tensor(Q, out, out_dtype)
     if want_lse and lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     st = lib.sparse_attn_fwd_dense(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
-                                   _ptr(lse), _stream(Q.device, stream))
+                                   SA_F32 if O.dtype == torch.float32 else SA_BF16, _ptr(lse),
+                                   _stream(Q.device, stream))
     _check("sparse_attn_fwd_dense", st)
     return (O, lse) if want_lse else O
 
@@ -229,6 +248,16 @@ def topk_count(k: float, n_k: int) -> int:
     if k >= 1.0:
         return n_k
     return min(n_k, max(0, math.ceil(k * n_k - 1e-9)))
+
+
+def exp2_poly_probe(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The attention kernel's software 2^x, evaluated on a CUDA fp32 tensor (test hook)."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 CUDA tensor")
+    y = torch.empty_like(x)
+    st = load_library().sparse_attn_test_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x.device, stream))
+    _check("sparse_attn_test_exp2_poly", st)
+    return y
 
 
 def version() -> str:

@@ -13,9 +13,10 @@
 #include <cuda_runtime.h>
 
 #include "sparse_attn.h"
+#include "sparse_attn_testing.h"
 #include "sa_ptx.cuh"
 #include "sa_mask_kernels.cuh"
-#include "sa_fwd_kernel.cuh"
+#include "sa_fwd2_kernel.cuh"
 
 namespace {
 
@@ -168,60 +169,88 @@ template <bool FROM_LOGITS>
 sa_status launch_select(const Dims& g, const float* in, int ld_in, double k, double p, int32_t* cnt,
                         int32_t* idx, uint8_t* mask, float* P_out, cudaStream_t st) {
     const int rows = g.BH * g.n_q;
-    const size_t smem = (size_t)sa::mask::SEL_WARPS * g.n_k * sizeof(uint32_t);
+    const int wpc = sa::mask::select_warps_per_cta(g.n_k);
+    const size_t smem = (size_t)wpc * 2 * g.n_k * sizeof(uint32_t);
     auto kern = sa::mask::select_kernel<FROM_LOGITS>;
     // Set on every call: the attribute is per device.
     sa_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  (int)((size_t)sa::mask::SEL_WARPS * MAX_NK * 4)),
+                                                  sa::mask::SEL_SMEM_BUDGET),
                              "select_kernel shared-memory attribute");
     if (s != SA_OK) return s;
-    const int grid = (rows + sa::mask::SEL_WARPS - 1) / sa::mask::SEL_WARPS;
-    kern<<<grid, sa::mask::SEL_WARPS * 32, smem, st>>>(in, ld_in, rows, g.n_k, topk_count(k, g.n_k),
-                                                        p, cnt, idx, mask, P_out);
+    const int grid = (rows + wpc - 1) / wpc;
+    kern<<<grid, wpc * 32, smem, st>>>(in, ld_in, rows, g.n_k, topk_count(k, g.n_k), p, cnt, idx, mask,
+                                       P_out);
     return cuda_check(cudaGetLastError(), "select_kernel launch");
 }
 
 template <int D, int BQ>
-sa_status launch_fwd_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
-                       const int32_t* idx, void* O, float* lse, bool dense, cudaStream_t st) {
-    using L = sa::fwd::SmemLayout<D>;
+sa_status launch_fwd2_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
+                        const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
+                        cudaStream_t st) {
+    using L = sa::fwd2::Layout2<D>;
     CUtensorMap mq, mk, mv;
     sa_status s;
-    if ((s = make_map(&mq, Q, g, sa::fwd::MROWS)) != SA_OK) return s;
-    if ((s = make_map(&mk, K, g, sa::fwd::BK)) != SA_OK) return s;
-    if ((s = make_map(&mv, V, g, sa::fwd::BK)) != SA_OK) return s;
-    auto kern = sa::fwd::sparse_fwd_kernel<D, BQ>;
+    if ((s = make_map(&mq, Q, g, sa::fwd2::MROWS)) != SA_OK) return s;
+    if ((s = make_map(&mk, K, g, sa::fwd2::BK)) != SA_OK) return s;
+    if ((s = make_map(&mv, V, g, sa::fwd2::BK)) != SA_OK) return s;
+    auto kern = sa::fwd2::sparse_fwd2_kernel<D, BQ>;
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
-                        "sparse_fwd_kernel shared-memory attribute")) != SA_OK)
+                        "sparse_fwd2_kernel shared-memory attribute")) != SA_OK)
         return s;
-    sa::fwd::FwdParams prm;
+    sa::fwd2::Fwd2Params prm;
     prm.cnt = cnt;
     prm.idx = idx;
-    prm.O = reinterpret_cast<__nv_bfloat16*>(O);
+    prm.O = O;
     prm.lse = lse;
     prm.N = g.N;
     prm.n_q = g.n_q;
     prm.n_k = g.n_k;
-    prm.bq = g.bq;
+    prm.rows = g.BH * g.n_q;
     prm.dense = dense ? 1 : 0;
+    prm.out_f32 = out_f32 ? 1 : 0;
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     prm.wait_limit_ns = WAIT_LIMIT_NS;
-    dim3 grid(g.n_q, g.BH);
-    kern<<<grid, sa::fwd::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, prm);
-    return cuda_check(cudaGetLastError(), "sparse_fwd_kernel launch");
+    const int grid = (prm.rows + sa::fwd2::NSLOT - 1) / sa::fwd2::NSLOT;
+    kern<<<grid, sa::fwd2::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, prm);
+    return cuda_check(cudaGetLastError(), "sparse_fwd2_kernel launch");
 }
 
 sa_status launch_fwd(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
-                     const int32_t* idx, void* O, float* lse, bool dense, cudaStream_t st) {
-    if (g.d == 128 && g.bq == 128) return launch_fwd_t<128, 128>(g, Q, K, V, cnt, idx, O, lse, dense, st);
-    if (g.d == 128 && g.bq == 64) return launch_fwd_t<128, 64>(g, Q, K, V, cnt, idx, O, lse, dense, st);
-    if (g.d == 64 && g.bq == 128) return launch_fwd_t<64, 128>(g, Q, K, V, cnt, idx, O, lse, dense, st);
-    return launch_fwd_t<64, 64>(g, Q, K, V, cnt, idx, O, lse, dense, st);
+                     const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
+                     cudaStream_t st) {
+    if (g.d == 128 && g.bq == 128)
+        return launch_fwd2_t<128, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+    if (g.d == 128 && g.bq == 64)
+        return launch_fwd2_t<128, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+    if (g.d == 64 && g.bq == 128)
+        return launch_fwd2_t<64, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+    return launch_fwd2_t<64, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+}
+
+sa_status check_out_dtype(int o_dtype) {
+    if (o_dtype != SA_BF16 && o_dtype != SA_F32)
+        return fail(SA_ERR_INVALID_ARG, "o_dtype=%d (SA_BF16=0 or SA_F32=1)", o_dtype);
+    return SA_OK;
+}
+
+__global__ void exp2_poly_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = sa::fwd2::exp2_poly(x[i]);
 }
 
 }  // namespace
 
 extern "C" {
+
+sa_status sparse_attn_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+    if (!x || !y || n < 0) return fail(SA_ERR_INVALID_ARG, "exp2 probe: bad arguments");
+    if (n == 0) return ok();
+    const int64_t blocks = (n + 255) / 256;
+    if (blocks > 0x7FFFFFFF) return fail(SA_ERR_INVALID_ARG, "exp2 probe: n too large");
+    exp2_poly_probe_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+    sa_status s = cuda_check(cudaGetLastError(), "exp2 probe launch");
+    return s != SA_OK ? s : ok();
+}
 
 size_t sparse_attn_mask_workspace_bytes(const sa_shape* shape) {
     Dims g;
@@ -269,32 +298,35 @@ sa_status sparse_attn_select(const sa_shape* shape, const float* P, double k, do
 }
 
 sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, const void* V,
-                          const int32_t* cnt, const int32_t* idx, void* O, float* lse_or_null,
-                          void* stream) {
+                          const int32_t* cnt, const int32_t* idx, void* O, int o_dtype,
+                          float* lse_or_null, void* stream) {
     Dims g;
     sa_status s;
     if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if ((s = check_out_dtype(o_dtype)) != SA_OK) return s;
     if (!Q || !K || !V || !cnt || !idx || !O)
         return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, cnt, idx, O");
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(cnt) || !aligned16(idx) ||
         !aligned16(O) || (lse_or_null && !aligned16(lse_or_null)))
         return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
-    s = launch_fwd(g, Q, K, V, cnt, idx, O, lse_or_null, false, reinterpret_cast<cudaStream_t>(stream));
+    s = launch_fwd(g, Q, K, V, cnt, idx, O, o_dtype == SA_F32, lse_or_null, false,
+                   reinterpret_cast<cudaStream_t>(stream));
     if (s != SA_OK) return s;
     return ok();
 }
 
 sa_status sparse_attn_fwd_dense(const sa_shape* shape, const void* Q, const void* K, const void* V,
-                                void* O, float* lse_or_null, void* stream) {
+                                void* O, int o_dtype, float* lse_or_null, void* stream) {
     Dims g;
     sa_status s;
     if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if ((s = check_out_dtype(o_dtype)) != SA_OK) return s;
     if (!Q || !K || !V || !O) return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, O");
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
         (lse_or_null && !aligned16(lse_or_null)))
         return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
     // The dense path reads no index list.
-    s = launch_fwd(g, Q, K, V, nullptr, nullptr, O, lse_or_null, true,
+    s = launch_fwd(g, Q, K, V, nullptr, nullptr, O, o_dtype == SA_F32, lse_or_null, true,
                    reinterpret_cast<cudaStream_t>(stream));
     if (s != SA_OK) return s;
     return ok();

@@ -183,48 +183,108 @@ __device__ __forceinline__ uint64_t fixed_mass(uint32_t bits) {
     return __float2ull_rz(__uint_as_float(bits) * 2147483648.0f);
 }
 
-// Sum of fixed-point mass over the row entries whose fp32 bit pattern is >= v.
-__device__ __forceinline__ uint64_t mass_at_least(const uint32_t* row, int n, uint32_t v, int lane) {
-    uint64_t s = 0;
-    for (int j = lane; j < n; j += 32) {
-        const uint32_t b = row[j];
-        if (b >= v) s += fixed_mass(b);
+// Boundary search over one score row held as fp32 bit patterns (P >= 0, so
+// unsigned order is numeric order). For the metric "fixed-point mass"
+// (MASS = true) or "number of entries" (MASS = false) it finds the largest
+// 31-bit value v such that the metric summed over the entries >= v still
+// reaches `target`, most significant bit first. The entries still able to
+// decide the answer (those inside the current range [v, v | (2^(b+1) - 1)])
+// are kept in `work` and compacted in place after every bit, so each step
+// only touches the survivors. Returns v and, through the out-parameters, the
+// count and mass of the entries strictly above v. Integer sums only: the
+// answer does not depend on the order of the reductions.
+struct Boundary {
+    uint32_t v;
+    int n_above;
+    uint64_t mass_above;
+};
+
+template <bool MASS>
+__device__ Boundary boundary_search(const uint32_t* __restrict__ bits, uint32_t* __restrict__ work,
+                                    int n, uint64_t target, int lane) {
+    for (int j = lane; j < n; j += 32) work[j] = bits[j];
+    __syncwarp();
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int m = n;
+    uint32_t v = 0;
+    int n_above = 0;
+    uint64_t mass_above = 0;
+    for (int b = 30; b >= 0; --b) {
+        const uint32_t bit = 1u << b;
+        uint64_t hi_mass = 0;
+        uint32_t hi_cnt = 0;
+        for (int j = lane; j < m; j += 32) {
+            const uint32_t x = work[j];
+            if (x & bit) {
+                ++hi_cnt;
+                if (MASS) hi_mass += fixed_mass(x);
+            }
+        }
+        hi_cnt = warp_sum_u32(hi_cnt);
+        if (MASS) hi_mass = warp_sum_u64(hi_mass);
+        const uint64_t reach = MASS ? mass_above + hi_mass : (uint64_t)(n_above + (int)hi_cnt);
+        const bool take = reach >= target;
+        if (take) {
+            v |= bit;  // entries without this bit fall below v
+        } else {
+            n_above += (int)hi_cnt;  // entries with this bit lie above the range
+            mass_above += hi_mass;
+        }
+        const int keep_n = take ? (int)hi_cnt : m - (int)hi_cnt;
+        if (keep_n != m) {
+            int out = 0;
+            for (int base = 0; base < m; base += 32) {
+                const int j = base + lane;
+                uint32_t x = 0;
+                bool keep = false;
+                if (j < m) {
+                    x = work[j];
+                    keep = ((x & bit) != 0) == take;
+                }
+                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
+                __syncwarp();
+                if (keep) work[out + __popc(bal & lt_mask)] = x;
+                out += __popc(bal);
+                __syncwarp();
+            }
+            m = keep_n;
+        }
     }
-    return warp_sum_u64(s);
+    if (!MASS) mass_above = 0;
+    return {v, n_above, mass_above};
 }
 
-__device__ __forceinline__ uint32_t count_at_least(const uint32_t* row, int n, uint32_t v, int lane) {
-    uint32_t c = 0;
-    for (int j = lane; j < n; j += 32) c += (row[j] >= v) ? 1u : 0u;
-    return warp_sum_u32(c);
+constexpr int SEL_MAX_WARPS = 4;
+constexpr int SEL_SMEM_BUDGET = 200 * 1024;
+
+// Warps (rows) per CTA of select_kernel for a row length n_k: each warp
+// holds its row twice in shared memory (8 bytes per entry).
+inline int select_warps_per_cta(int n_k) {
+    int w = SEL_SMEM_BUDGET / (8 * n_k);
+    return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : w);
 }
 
-constexpr int SEL_WARPS = 4;
-
-// One warp per score row. The row's scores are kept in shared memory as fp32
-// bit patterns; P >= 0, so comparing bit patterns as unsigned integers orders
-// the scores exactly.
-//
-// The kept set is the first L entries of the order "score descending, then
-// index ascending", L = max(kc, m_p):
+// One warp per score row. The kept set is the first L entries of the order
+// "score descending, then index ascending", L = max(kc, m_p):
 //   kc  = number of Top-k blocks (computed on the host);
 //   m_p = shortest prefix whose fixed-point mass reaches T = ceil(p * W).
-// Both boundaries are found by a most-significant-bit-first search over the
-// 31 value bits of the score (the largest threshold v whose "entries >= v"
-// still have enough mass, or enough entries), then resolved inside the group
-// of entries equal to the boundary score by index order. Every quantity is an
-// integer count or an integer sum, so the result does not depend on the
-// order of the reductions and equals a full sort's prefix bit for bit.
+// m_p comes from the mass boundary v (entries above v, then as many of the
+// entries equal to v as the remaining mass needs); if kc is larger, the
+// count boundary of kc is searched the same way. The kept indices are then
+// written in ascending order, ties at the boundary taken by lower index.
+// The result equals the prefix of a full sort bit for bit.
 template <bool FROM_LOGITS>
-__global__ void __launch_bounds__(SEL_WARPS * 32)
+__global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
 select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
               int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
               float* __restrict__ P_out) {
     extern __shared__ uint32_t sel_smem[];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const long long row = (long long)blockIdx.x * SEL_WARPS + warp;
+    const int wpc = blockDim.x / 32;
+    const long long row = (long long)blockIdx.x * wpc + warp;
     if (row >= n_rows) return;
-    uint32_t* bits = sel_smem + (size_t)warp * n_k;
+    uint32_t* bits = sel_smem + (size_t)warp * 2 * n_k;
+    uint32_t* work = bits + n_k;
     const float* src = in + (size_t)row * ld_in;
 
     if (FROM_LOGITS) {
@@ -257,8 +317,11 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
     }
     __syncwarp();
 
-    // L = number of kept entries.
-    int L;
+    // L = number of kept entries; (v, n_above) = its boundary score and the
+    // number of entries strictly above it.
+    int L = kc;
+    bool have_boundary = false;
+    Boundary bd = {0u, 0, 0ull};
     if (p >= 1.0) {
         L = n_k;
     } else {
@@ -266,20 +329,17 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
         for (int j = lane; j < n_k; j += 32) w += fixed_mass(bits[j]);
         const uint64_t W = warp_sum_u64(w);
         const uint64_t T = (uint64_t)ceil(p * (double)W);
-        int m_p = 0;
         if (T > 0) {
-            uint32_t v = 0;
-            for (int bit = 30; bit >= 0; --bit) {
-                const uint32_t cand = v | (1u << bit);
-                if (mass_at_least(bits, n_k, cand, lane) >= T) v = cand;
+            const Boundary mb = boundary_search<true>(bits, work, n_k, T, lane);
+            const uint64_t wb = fixed_mass(mb.v);  // > 0 for scores in [0, 1]
+            const uint64_t need = wb ? (T - mb.mass_above + wb - 1) / wb : 1;
+            const int m_p = (int)(mb.n_above + need);
+            if (m_p >= kc) {
+                L = m_p;
+                bd = mb;
+                have_boundary = true;
             }
-            const uint64_t above = mass_at_least(bits, n_k, v + 1u, lane);
-            const uint32_t n_above = count_at_least(bits, n_k, v + 1u, lane);
-            const uint64_t wb = fixed_mass(v);  // > 0 for scores in [0, 1]
-            const uint64_t need = wb ? (T - above + wb - 1) / wb : 1;
-            m_p = (int)(n_above + need);
         }
-        L = max(kc, m_p);
     }
     L = min(L, n_k);
 
@@ -290,18 +350,14 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
             idx_row[j] = j;
             if (mask_row) mask_row[j] = 1;
         }
-    } else if (L == 0) {
+    } else if (L <= 0) {
+        L = 0;
         if (mask_row)
             for (int j = lane; j < n_k; j += 32) mask_row[j] = 0;
     } else {
-        // Boundary score for L entries, then how many of its ties are kept.
-        uint32_t v = 0;
-        for (int bit = 30; bit >= 0; --bit) {
-            const uint32_t cand = v | (1u << bit);
-            if ((int)count_at_least(bits, n_k, cand, lane) >= L) v = cand;
-        }
-        const int n_above = (int)count_at_least(bits, n_k, v + 1u, lane);
-        const int ties_kept = L - n_above;
+        if (!have_boundary) bd = boundary_search<false>(bits, work, n_k, (uint64_t)L, lane);
+        const uint32_t v = bd.v;
+        const int ties_kept = L - bd.n_above;
         int ties_before = 0, kept_before = 0;
         const uint32_t lt_mask = (1u << lane) - 1u;
         for (int base = 0; base < n_k; base += 32) {

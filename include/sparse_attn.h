@@ -20,7 +20,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Tensors are dense, row-major, with no padding:
- *     Q, K, V, O   bf16  [B, H, N, d]     (token-major within a head)
+ *     Q, K, V      bf16  [B, H, N, d]     (token-major within a head)
+ *     O            bf16 or fp32 [B, H, N, d]
  *     cnt          int32 [B, H, n_q]
  *     idx          int32 [B, H, n_q, n_k] (row capacity n_k)
  *     mask         uint8 [B, H, n_q, n_k]
@@ -63,6 +64,12 @@ typedef enum {
 typedef struct {
     int32_t B, H, N, d, bq, bk;
 } sa_shape;
+
+/* Element type of the attention output O. */
+typedef enum {
+    SA_BF16 = 0,  /* bf16, the fp32 result rounded to nearest even */
+    SA_F32 = 1    /* fp32, the kernel's result before that rounding */
+} sa_dtype;
 
 /* Bytes of device workspace sparse_attn_mask needs for `shape` (pooled Q and
  * K, and the fp32 block-logit matrix). 0 on an invalid shape. */
@@ -109,15 +116,19 @@ sa_status sparse_attn_select(const sa_shape* shape, const float* P, double k, do
  * O = 0 and lse = -inf. Index entries must lie in [0, n_k); an entry outside
  * is skipped and reported as SA_ERR_DEVICE_ASSERT.
  * Inputs: Q, K, V bf16 [B,H,N,d]; cnt, idx as produced by sparse_attn_mask.
- * Outputs: O bf16 [B,H,N,d]; lse (optional) fp32 [B,H,N]. */
+ * Outputs: O [B,H,N,d] of type o_dtype (SA_BF16 or SA_F32; the bf16 output
+ *          is exactly the round-to-nearest-even of the fp32 one);
+ *          lse (optional) fp32 [B,H,N], natural log of the softmax
+ *          denominator of each query row. */
 sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, const void* V,
                           const int32_t* cnt, const int32_t* idx,
-                          void* O, float* lse_or_null, void* stream);
+                          void* O, int o_dtype, float* lse_or_null, void* stream);
 
 /* Step 4 with every key block kept (full attention through the same kernel;
  * no index list is read). The reference point for the sparse speed-up. */
 sa_status sparse_attn_fwd_dense(const sa_shape* shape, const void* Q, const void* K,
-                                const void* V, void* O, float* lse_or_null, void* stream);
+                                const void* V, void* O, int o_dtype, float* lse_or_null,
+                                void* stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (SA_OK if none) and clears the record. */

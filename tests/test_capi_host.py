@@ -8,7 +8,7 @@ import re
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "sparse_attn.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("sparse_attn.h", "sparse_attn_testing.h")]
 
 
 @pytest.fixture(scope="module")
@@ -20,8 +20,10 @@ def lib():
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(sparse_attn_\w+)\s*\(", src)))
+    names = set()
+    for h in HEADERS:
+        names |= set(re.findall(r"\b(sparse_attn_\w+)\s*\(", open(h).read()))
+    return sorted(names)
 
 
 def test_header_declares_the_binding_list():
@@ -80,8 +82,11 @@ def test_host_validation_codes(lib):
     assert _mask_status(lib, good, ptr=8) == 1           # misaligned
     assert b"aligned" in lib.sparse_attn_last_error()
     z = ctypes.c_void_p(0)
-    assert lib.sparse_attn_fwd(good, z, z, z, z, z, z, None, None) == 1
-    assert lib.sparse_attn_fwd_dense(good, z, z, z, z, None, None) == 1
+    assert lib.sparse_attn_fwd(good, z, z, z, z, z, z, 0, None, None) == 1
+    assert lib.sparse_attn_fwd_dense(good, z, z, z, z, 0, None, None) == 1
+    a = ctypes.c_void_p(16)
+    assert lib.sparse_attn_fwd(good, a, a, a, a, a, a, 7, None, None) == 1   # unknown o_dtype
+    assert b"o_dtype" in lib.sparse_attn_last_error()
     assert lib.sparse_attn_select(good, z, 0.1, 0.9, z, z, None, None) == 1
     assert lib.sparse_attn_select(good, ctypes.c_void_p(16), 0.0, 0.0, ctypes.c_void_p(16),
                                   ctypes.c_void_p(16), None, None) == 1
@@ -101,3 +106,21 @@ def test_topk_count_matches_oracle_rule():
     for k in (0.0, 0.03, 0.05, 0.07, 0.1, 0.125, 0.25, 0.5, 0.999, 1.0):
         for n in (1, 7, 64, 100, 256, 275, 512, 1182):
             assert topk_count(k, n) == oracle.topk_count(k, n)
+
+
+def test_exp2_poly_constants_come_from_the_remez_script():
+    """The kernel's polynomial constants are the ones the derivation script prints."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "gen_exp2_poly", os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "gen_exp2_poly.py"))
+    gen = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(gen)
+    coef, err = gen.remez_relative()
+    assert err < 1e-4
+    src = open(os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "sa_fwd2_kernel.cuh")).read()
+    body = src[src.index("float exp2_poly("):src.index("return (x == -INFINITY)")]
+    lits = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[-+][0-9]+)f", body)]
+    assert len(lits) == 4
+    c3, c2, c1, c0 = lits
+    import numpy as np
+    assert np.allclose([c0, c1, c2, c3], np.float32(coef), rtol=0, atol=2e-9)

@@ -2,7 +2,10 @@
 
 Both sides use the GPU's own mask, so selection near-ties do not enter the
 output comparison. Tolerance for bf16 inputs against the fp64 oracle:
-max-abs 1e-2 and mean-abs 1e-3.
+max-abs 1e-2 and mean-abs 1e-3, on the kernel's fp32 result (SA_F32). The
+bf16 output (SA_BF16) must be exactly that result rounded to nearest even:
+the final rounding alone is up to half a bf16 ulp, 2^-8 |O|, which for
+|O| >= 2.56 exceeds 1e-2 by itself.
 """
 import numpy as np
 import pytest
@@ -23,8 +26,11 @@ pytestmark = pytest.mark.gpu
 def _run(name, k, p, rows_stride=None):
     cfg, (Q, K, V), (Qh, Kh, Vh) = workload(name)
     m = sparse_attn_mask(Q, K, cfg.bq, cfg.bk, k, p)
-    O_gpu, lse = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], cfg.bq, cfg.bk, want_lse=True)
+    O_gpu, lse = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], cfg.bq, cfg.bk, want_lse=True,
+                                 out_dtype=torch.float32)
+    O_bf16 = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], cfg.bq, cfg.bk)
     check_device_error(Q.device)
+    assert torch.equal(O_bf16, O_gpu.to(torch.bfloat16))
     cnt = m["cnt"].cpu().numpy()
     idx = m["idx"].cpu().numpy()
     rows = all_rows(cfg.B, cfg.H, cfg.n_q) if rows_stride is None else \
@@ -45,7 +51,7 @@ def test_fwd_matches_oracle(name, stride):
     cfg = CONFIGS[name]
     mx, mean, lerr = _run(name, cfg.k, cfg.p, stride)
     assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL
-    assert lerr < 1e-3
+    assert lerr < 1e-4
 
 
 @pytest.mark.parametrize("k,p", [(0.03, 0.80), (0.05, 0.90), (0.10, 0.95)])
@@ -66,8 +72,10 @@ def test_fwd_ragged_shapes(N, d, bq, k, p):
     B, H = 2, 3
     Q, K, V, Qh, Kh, Vh = _custom_case(B, H, N, d, bq, seed=7 * N + d, positional_field=True)
     m = sparse_attn_mask(Q, K, bq, 64, k, p)
-    O_gpu = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, 64)
+    O_gpu = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, 64, out_dtype=torch.float32)
+    O_bf16 = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, 64)
     check_device_error()
+    assert torch.equal(O_bf16, O_gpu.to(torch.bfloat16))
     n_q = -(-N // bq)
     rows = all_rows(B, H, n_q)
     O_ref, _ = O.block_sparse_attention(Qh, Kh, Vh, m["cnt"].cpu().numpy(), m["idx"].cpu().numpy(),
@@ -99,7 +107,7 @@ def test_fwd_arbitrary_lists_empty_rows_and_odd_counts(N, d, bq):
     n_q, n_k = -(-N // bq), -(-N // 64)
     cnt, idx = _handmade_lists(B, H, n_q, n_k, rng)
     O_gpu, lse = sparse_attn_fwd(Q, K, V, torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(),
-                                 bq, 64, want_lse=True)
+                                 bq, 64, want_lse=True, out_dtype=torch.float32)
     check_device_error()
     rows = all_rows(B, H, n_q)
     O_ref, L_ref = O.block_sparse_attention(Qh, Kh, Vh, cnt, idx, bq, 64, rows=rows)
@@ -119,7 +127,8 @@ def test_fwd_bad_index_is_reported_and_skipped():
     idx = np.zeros((B, H, n_q, n_k), dtype=np.int32)
     idx[..., :3] = [1, 4, 7]
     idx[0, 1, 2, 1] = n_k + 5                       # out of range: skipped, reported
-    O_gpu = sparse_attn_fwd(Q, K, V, torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(), bq, 64)
+    O_gpu = sparse_attn_fwd(Q, K, V, torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(), bq, 64,
+                            out_dtype=torch.float32)
     with pytest.raises(SparseAttnError, match="SA_ERR_DEVICE_ASSERT"):
         check_device_error()
     check_device_error()
@@ -135,7 +144,7 @@ def test_fwd_bad_index_is_reported_and_skipped():
 @pytest.mark.parametrize("name", ["tiny", "mid"])
 def test_dense_path_matches_torch_fp32_sdpa(name):
     cfg, (Q, K, V), _ = workload(name)
-    O_gpu = sparse_attn_fwd_dense(Q, K, V, cfg.bq, cfg.bk)
+    O_gpu = sparse_attn_fwd_dense(Q, K, V, cfg.bq, cfg.bk, out_dtype=torch.float32)
     check_device_error()
     ref = torch.nn.functional.scaled_dot_product_attention(Q.float(), K.float(), V.float())
     err = (O_gpu.float() - ref).abs()
@@ -159,3 +168,17 @@ def test_fwd_is_deterministic():
     b = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], cfg.bq, cfg.bk)
     check_device_error()
     assert torch.equal(a, b)
+
+
+def test_software_exp2_within_its_bound():
+    """The FMA-pipe 2^x used for a quarter of the softmax: relative error < 1e-4
+    over the arguments the kernel produces (x <= 8), exact 0 at -inf."""
+    from block_sparse_attention_row_b200.capi import exp2_poly_probe
+    x = torch.cat([torch.linspace(-124.0, 8.0, 2_000_001, dtype=torch.float64),
+                   torch.tensor([0.0, -0.5, 0.5, -1e-30, 8.0, -20.25])]).float().cuda()
+    y = exp2_poly_probe(x).double()
+    ref = torch.exp2(x.double())
+    rel = ((y - ref).abs() / ref).max().item()
+    assert rel < 1e-4, rel
+    z = exp2_poly_probe(torch.tensor([-float("inf")], device="cuda"))
+    assert z.item() == 0.0

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
                 4: "SA_ERR_TIMEOUT", 5: "SA_ERR_DEVICE_ASSERT"}
 
 # Every entry point declared in include/sparse_attn.h and include/sparse_attn_testing.h.
-EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_select",
+EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_mask_noalloc",
+            "sparse_attn_select",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_exp2_poly")
 
@@ -61,6 +62,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_mask.argtypes = [sp, vp, vp, ctypes.c_double, ctypes.c_double, i32p, i32p,
                                          u8p, f32p, vp, vp]
         lib.sparse_attn_mask.restype = ctypes.c_int
+        lib.sparse_attn_mask_noalloc.argtypes = [sp, vp, vp, ctypes.c_double, ctypes.c_double, i32p,
+                                                 i32p, u8p, f32p, vp]
+        lib.sparse_attn_mask_noalloc.restype = ctypes.c_int
         lib.sparse_attn_select.argtypes = [sp, f32p, ctypes.c_double, ctypes.c_double, i32p, i32p,
                                            u8p, vp]
         lib.sparse_attn_select.restype = ctypes.c_int
@@ -151,6 +155,30 @@ def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: floa
                               _ptr(res.get("P")), _ptr(workspace), _stream(dev, stream))
     _check("sparse_attn_mask", st)
     return res
+
+
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def sparse_attn_mask_noalloc(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: float,
+                             p: float, *, out: dict, stream=None) -> dict:
+    """sparse_attn_mask for callers that cannot allocate device memory on the call path.
+
+    The library uses its own fixed 32 MiB device scratch instead of a workspace,
+    so this call allocates nothing: the caller passes every output in `out`
+    ('cnt', 'idx', and optionally 'mask' and 'P', shaped as for
+    sparse_attn_mask). Shapes needing a larger workspace are rejected. Calls
+    that run concurrently on the GPU share the scratch and must not overlap.
+    """
+    _check_qkv(Q, K)
+    lib = load_library()
+    B, H, N, d = Q.shape
+    shape = make_shape(B, H, N, d, bq, bk)
+    st = lib.sparse_attn_mask_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(K), float(k), float(p),
+                                      _ptr(out["cnt"]), _ptr(out["idx"]), _ptr(out.get("mask")),
+                                      _ptr(out.get("P")), _stream(Q.device, stream))
+    _check("sparse_attn_mask_noalloc", st)
+    return out
 
 
 def sparse_attn_select(P: torch.Tensor, N: int, d: int, bq: int, bk: int, k: float, p: float, *,

@@ -282,6 +282,63 @@ sa_status sparse_attn_mask(const sa_shape* shape, const void* Q, const void* K, 
     return ok();
 }
 
+}  // extern "C"
+
+// ------------------------------------------------- allocation-free mask
+// The scratch of sparse_attn_mask_noalloc: a fixed device array, one per
+// device that loads this library, alive until the process exits. In host
+// code `g_noalloc_scratch` is only a stand-in for the symbol, never a device
+// address: kernels get the address that cudaGetSymbolAddress returns for the
+// current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SPARSE_ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (with that device current) and cached.
+sa_status noalloc_scratch(void** out) {
+    int dev = -1;
+    sa_status s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+    if (s != SA_OK) return s;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES)
+        return fail(SA_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, NOALLOC_MAX_DEVICES);
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        s = cuda_check(cudaGetSymbolAddress(&ptr, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+        if (s != SA_OK) return s;
+        if (!ptr) return fail(SA_ERR_CUDA, "scratch array has no device address");
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sa_status sparse_attn_mask_noalloc(const sa_shape* shape, const void* Q, const void* K, double k,
+                                   double p, int32_t* cnt, int32_t* idx, uint8_t* mask_or_null,
+                                   float* P_out_or_null, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    const size_t need = workspace_layout(g).total;
+    if (need > (size_t)SPARSE_ATTN_NOALLOC_SCRATCH_BYTES)
+        return fail(SA_ERR_UNSUPPORTED,
+                    "workspace of %zu bytes exceeds the %u-byte scratch of sparse_attn_mask_noalloc; "
+                    "use sparse_attn_mask with a caller-provided workspace",
+                    need, (unsigned)SPARSE_ATTN_NOALLOC_SCRATCH_BYTES);
+    void* scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != SA_OK) return s;
+    return sparse_attn_mask(shape, Q, K, k, p, cnt, idx, mask_or_null, P_out_or_null, scratch, stream);
+}
+
 sa_status sparse_attn_select(const sa_shape* shape, const float* P, double k, double p, int32_t* cnt,
                              int32_t* idx, uint8_t* mask_or_null, void* stream) {
     Dims g;

@@ -101,6 +101,30 @@ sa_status sparse_attn_mask(const sa_shape* shape, const void* Q, const void* K,
                            uint8_t* mask_or_null, float* P_out_or_null,
                            void* workspace, void* stream);
 
+/* sparse_attn_mask without a caller-provided workspace, for callers that
+ * cannot allocate device memory on their call path: for example a runtime
+ * that has handed all device memory to its own pool, or a plugin or callback
+ * context where a cudaMalloc is not allowed or would stall the device. It has
+ * no counterpart in the papers; it is a packaging of the same computation.
+ * Same arguments, outputs and selection as sparse_attn_mask, minus the
+ * workspace. The scratch lives in one fixed device array inside the library,
+ * SPARSE_ATTN_NOALLOC_SCRATCH_BYTES (32 MiB) per device, held by every GPU
+ * that loads the library until the process exits. Shapes whose workspace
+ * (sparse_attn_mask_workspace_bytes) exceeds it are rejected with
+ * SA_ERR_UNSUPPORTED before anything is enqueued. The function allocates
+ * nothing. The first call on a device looks up the array's device address
+ * (a runtime call), so make that first call before any stream capture. All
+ * calls share the array: calls whose work overlaps on the GPU (different
+ * streams, or different host threads, without ordering between them) race
+ * on it and give undefined results. Nothing in the array needs clearing:
+ * each call writes every scratch byte it later reads. */
+#define SPARSE_ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+sa_status sparse_attn_mask_noalloc(const sa_shape* shape, const void* Q, const void* K,
+                                   double k, double p,
+                                   int32_t* cnt, int32_t* idx,
+                                   uint8_t* mask_or_null, float* P_out_or_null,
+                                   void* stream);
+
 /* Step 3 alone, on a caller-supplied fp32 score matrix P [B,H,n_q,n_k]
  * (rows of non-negative finite values). Same selection code and outputs as
  * sparse_attn_mask; used to check the selection bit for bit. */

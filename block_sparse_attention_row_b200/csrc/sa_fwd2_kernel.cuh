@@ -10,20 +10,22 @@
 //
 // One CTA serves two query-block rows ("slots") at once so that the tensor
 // cores always have one slot's matmuls to run while the other slot's softmax
-// is computed. 320 threads in four roles:
-//   warp 0      TMA producer: each slot's Q tile once, then K and V chunks
+// is computed. 384 threads in four roles:
+//   warp 8      TMA producer: each slot's Q tile once, then K and V chunks
 //               (two kept key blocks = 128 keys per chunk) gathered by the
 //               slots' index lists into a ring of 32 KB chunks, in a fixed
 //               interleaved order both the producer and the MMA issuer walk;
-//   warp 1      tcgen05 issuer (one thread): S_s = Q_s K^T into TMEM, then
+//   warp 9      tcgen05 issuer (one thread): S_s = Q_s K^T into TMEM, then
 //               O_s += P_s V with P_s read from TMEM where the softmax wrote it
 //               over S_s (the next S_s is issued after that product, and the
 //               tensor pipe executes one thread's MMAs in order);
-//   warps 2-5   softmax of slot 0, warps 6-9 softmax of slot 1: one query row
+//   warps 0-3   softmax of slot 0, warps 4-7 softmax of slot 1: one query row
 //               per thread (one TMEM lane), base-2 online softmax with a lazy
 //               rescale of O (only when the running max grows by more than
 //               2^8); a quarter of the exponentials run as a polynomial on the
 //               FMA pipe to offload the MUFU unit; then the epilogue.
+//   warps 10-11 idle. The control warpgroup (8-11) hands most of its
+//               registers to the two softmax warpgroups (setmaxnreg).
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d),
 // O_1 [384,384+d); P_s (bf16 pairs) overwrites the first 64 columns of S_s.
 // Tensor-core shapes: S tile M=128 x N=128 x K=d (A, B from shared memory);
@@ -42,9 +44,24 @@ constexpr int BK = 64;           // key block (tokens)
 constexpr int TILE_N = 128;      // keys per chunk: two kept key blocks
 constexpr int MROWS = 128;       // query rows per MMA tile
 constexpr int NSLOT = 2;         // query-block rows per CTA
-constexpr int NUM_THREADS = 64 + NSLOT * 128;
+constexpr int NUM_THREADS = 384;   // softmax warpgroups 0-1, control warpgroup 2
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+// Register split (setmaxnreg): the kernel launches with LAUNCH_REGS per thread
+// (384 x 168 = 64512 registers); the control warpgroup gives back down to
+// CTRL_REGS and the two softmax warpgroups take the rest:
+// 128 x 40 + 256 x 232 = 64512.
+constexpr int LAUNCH_REGS = 168;
+constexpr int CTRL_REGS = 40;
+constexpr int SOFTMAX_REGS = 232;
+static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= NUM_THREADS * LAUNCH_REGS, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float LAZY_RESCALE_LOG2 = 8.0f;
+// One column pair in EXP_POLY_EVERY takes its exponentials on the FMA pipe
+// (exp2_poly) instead of the MUFU unit; 0 keeps every exponential on MUFU.
+// Measured on B200: the MUFU unit is not the limit of this kernel, and the
+// polynomial's extra instructions lengthen the softmax, so it is off.
+constexpr int EXP_POLY_EVERY = 0;
 constexpr int MAX_CHUNKS = 10;
 
 // Where a bounded wait gave up (reported in the device error record).
@@ -139,14 +156,39 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t y, float& r0, float& r1)
     r1 = (y1 == -INFINITY) ? 0.f : r1;
 }
 
-// O[d_tmem] (+)= A[TMEM] * B[smem desc], bf16, fp32 accumulate.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate) {
+// The MMA issuer keeps each shared-memory descriptor as a (low, high) word
+// pair: moving the start address by a byte offset adds offset >> 4 to the
+// low word (offsets stay below 2^18 bytes, so the 14-bit field never
+// carries), which keeps the instructions between two MMAs to a minimum.
+struct Desc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ Desc desc_split(uint64_t d) {
+    return {static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+
+// D[tmem] (+)= A[smem] * B[smem], bf16, fp32 accumulate; descriptors as word pairs.
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, Desc a, uint32_t a_off16, Desc b,
+                                        uint32_t b_off16, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+        "mov.b64 ad, {%1, %2};\n\t"
+        "mov.b64 bd, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a.lo + a_off16), "r"(a.hi), "r"(b.lo + b_off16), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// O[d_tmem] (+)= A[TMEM] * B[smem desc], bf16, fp32 accumulate.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, Desc b, uint32_t b_off16,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b.lo + b_off16), "r"(b.hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -227,7 +269,7 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         fence_mbarrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         tmem_alloc(&C.tmem_base, TMEM_COLS);
         tmem_relinquish();
     }
@@ -237,7 +279,10 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t tmem = C.tmem_base;
     const uint64_t lim = prm.wait_limit_ns;
 
-    if (warp == 0) {
+    if (warp >= 2 * 4) {
+      // Control warpgroup: producer, MMA issuer, two idle warps.
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(CTRL_REGS));
+      if (warp == PRODUCER_WARP) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_descriptor(&tmQ);
@@ -304,13 +349,14 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == MMA_WARP) {
         // ----------------------------------------------------- MMA issuer
         if (lane == 0 && (nt[0] > 0 || nt[1] > 0)) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(MROWS, TILE_N, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(MROWS, D, true);
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t ch_addr = smem_u32(sCH);
+            const Desc q_desc = desc_split(kmajor_desc(smem_u32(sQ)));
+            const Desc k_desc = desc_split(kmajor_desc(smem_u32(sCH)));
+            const Desc v_desc = desc_split(mnmajor_desc(smem_u32(sCH), TILE_N * 128));
             bool ok = true;
             for (int s = 0; s < NSLOT && ok; ++s)
                 if (nt[s] > 0) ok = mbar_wait_bounded(&C.q_full[s], 0, abort_flag, W_Q, lim);
@@ -322,18 +368,19 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         ok = false;
                         return false;
                     }
-                    const uint32_t cb = ch_addr + c * L::CH_BYTES;
+                    const uint32_t c16 = (uint32_t)(c * L::CH_BYTES) >> 4;  // chunk offset, 16-byte units
                     const uint32_t tS = tmem + s * TILE_N;
                     if (!is_v) {
                         tc_fence_after();
-                        const uint32_t qb = q_addr + s * L::Q_BYTES;
+                        const Desc qd = {q_desc.lo + ((uint32_t)(s * L::Q_BYTES) >> 4), q_desc.hi};
+                        const Desc kd = {k_desc.lo + c16, k_desc.hi};
 #pragma unroll
                         for (int sl = 0; sl < L::SLABS; ++sl) {
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
-                                const uint64_t a = kmajor_desc(qb + sl * (MROWS * 128) + kk * 32);
-                                const uint64_t b = kmajor_desc(cb + sl * (TILE_N * 128) + kk * 32);
-                                umma_bf16(tS, a, b, IDESC_S, (sl > 0 || kk > 0) ? 1u : 0u);
+                                umma_ss(tS, qd, (sl * (MROWS * 128) + kk * 32) >> 4, kd,
+                                        (sl * (TILE_N * 128) + kk * 32) >> 4, IDESC_S,
+                                        (sl > 0 || kk > 0) ? 1u : 0u);
                             }
                         }
                         umma_commit(&C.s_full[s]);
@@ -345,10 +392,11 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                         }
                         tc_fence_after();
                         const uint32_t tO = tmem + 2 * TILE_N + s * TILE_N;
+                        const Desc vd = {v_desc.lo + c16, v_desc.hi};
 #pragma unroll
                         for (int kk = 0; kk < TILE_N / 16; ++kk) {
-                            const uint64_t b = mnmajor_desc(cb + kk * 16 * 128, TILE_N * 128);
-                            umma_bf16_ts(tO, tS + kk * 8, b, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                            umma_ts(tO, tS + kk * 8, vd, (kk * 16 * 128) >> 4, IDESC_PV,
+                                    (t > 0 || kk > 0) ? 1u : 0u);
                         }
                         umma_commit(&C.ch_empty[c]);
                         if (t == nt[s] - 1) umma_commit(&C.o_done[s]);
@@ -365,9 +413,11 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
             }
         }
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SOFTMAX_REGS));
         // ------------------------------------------- softmax and epilogue
-        const int s = (warp - 2) / 4;            // slot of this warpgroup
+        const int s = warp / 4;                  // slot of this warpgroup
         const int wq = warp & 3;                 // TMEM lane quarter of this warp
         const int row = wq * 32 + lane;          // query row within the tile
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -379,22 +429,24 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const bool row_valid = (row < BQ) && (q_tok < prm.N) && (blockIdx.x * NSLOT + s < prm.rows);
         const float sl2 = prm.scale_log2;
         const int32_t* lst = idx_row[s];
-        auto block_at = [&](int e) -> int {
+        // Index-list entries are loaded a tile ahead and range-checked only
+        // when used, so the load latency hides behind a tile of work.
+        auto block_raw = [&](int e) -> int {
             if (e >= cnt) return -1;
-            const int j = prm.dense ? e : __ldg(lst + e);
-            return (j >= 0 && j < n_k) ? j : -1;
+            return prm.dense ? e : __ldg(lst + e);
         };
+        auto checked = [&](int j) -> int { return (j >= 0 && j < n_k) ? j : -1; };
         const bool want_lse = prm.lse != nullptr;
         float m_run = -INFINITY;  // running max, log2 units, as used for P
         float l_run = 0.f;        // sum of the bf16-rounded weights: normalises O
         float l_exact = 0.f;      // sum of the unrounded weights: the log-sum-exp
         bool ok = true;
-        int nj0 = my_nt > 0 ? block_at(0) : -1, nj1 = my_nt > 0 ? block_at(1) : -1;
+        int nj0 = my_nt > 0 ? block_raw(0) : -1, nj1 = my_nt > 0 ? block_raw(1) : -1;
         for (int t = 0; t < my_nt; ++t) {
-            const int j0 = nj0, j1 = nj1;
+            const int j0 = checked(nj0), j1 = checked(nj1);
             if (t + 1 < my_nt) {  // next tile's blocks, loaded while this one is computed
-                nj0 = block_at(2 * t + 2);
-                nj1 = block_at(2 * t + 3);
+                nj0 = block_raw(2 * t + 2);
+                nj1 = block_raw(2 * t + 3);
             }
             const bool w = mbar_wait_bounded(&C.s_full[s], t & 1, abort_flag, W_S_FULL, lim);
             if (!__all_sync(0xFFFFFFFFu, w)) {
@@ -442,28 +494,32 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[q] = 0ull;
             acc_exact[0] = acc_exact[1] = 0ull;
-            uint32_t pk[TILE_N / 2];
 #pragma unroll
-            for (int c = 0; c < TILE_N / 2; ++c) {
-                // y = S * log2(e)/sqrt(d) - m for two columns at once.
-                const uint64_t y = f2_fma(f2_pack(__uint_as_float(r[2 * c]), __uint_as_float(r[2 * c + 1])),
-                                          scale2, negm2);
-                float p0, p1;
-                if ((c & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
-                    exp2_poly_pair(y, p0, p1);
-                } else {
-                    float y0, y1;
-                    f2_unpack(y, y0, y1);
-                    p0 = ex2_approx(y0);
-                    p1 = ex2_approx(y1);
+            for (int h = 0; h < 2; ++h) {  // two halves of 64 keys: P columns [32h, 32h + 32)
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int pc = 32 * h + c;  // column pair
+                    // y = S * log2(e)/sqrt(d) - m for two columns at once.
+                    const uint64_t y = f2_fma(f2_pack(__uint_as_float(r[2 * pc]), __uint_as_float(r[2 * pc + 1])),
+                                              scale2, negm2);
+                    float p0, p1;
+                    if (EXP_POLY_EVERY > 0 && pc % (EXP_POLY_EVERY > 0 ? EXP_POLY_EVERY : 1) == EXP_POLY_EVERY - 1) {
+                        exp2_poly_pair(y, p0, p1);
+                    } else {
+                        float y0, y1;
+                        f2_unpack(y, y0, y1);
+                        p0 = ex2_approx(y0);
+                        p1 = ex2_approx(y1);
+                    }
+                    pk[c] = pack_bf16x2(p0, p1);
+                    // Sum the bf16-rounded weights the PV product uses.
+                    acc[c & 3] = f2_add(acc[c & 3], f2_pack(__uint_as_float(pk[c] << 16),
+                                                            __uint_as_float(pk[c] & 0xFFFF0000u)));
+                    if (want_lse) acc_exact[c & 1] = f2_add(acc_exact[c & 1], f2_pack(p0, p1));
                 }
-                pk[c] = pack_bf16x2(p0, p1);
-                // Sum the bf16-rounded weights the PV product uses.
-                acc[c & 3] = f2_add(acc[c & 3], f2_pack(__uint_as_float(pk[c] << 16),
-                                                        __uint_as_float(pk[c] & 0xFFFF0000u)));
-                if (want_lse) acc_exact[c & 1] = f2_add(acc_exact[c & 1], f2_pack(p0, p1));
+                tmem_st32_nowait(tS + 32 * h, pk);
             }
-            tmem_st64_nowait(tS, pk);
             {
                 const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
                 float a0, a1;
@@ -536,7 +592,7 @@ sparse_fwd2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
 
     __syncthreads();
-    if (warp == 1) {
+    if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

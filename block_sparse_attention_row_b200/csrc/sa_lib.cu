@@ -197,6 +197,13 @@ sa_status launch_fwd2_t(const Dims& g, const void* Q, const void* K, const void*
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
                         "sparse_fwd2_kernel shared-memory attribute")) != SA_OK)
         return s;
+    // The kernel moves registers between its warpgroups (setmaxnreg); the
+    // split adds up only for the launch register count it was written for.
+    cudaFuncAttributes fa;
+    if ((s = cuda_check(cudaFuncGetAttributes(&fa, kern), "sparse_fwd2_kernel attributes")) != SA_OK) return s;
+    if (fa.numRegs != sa::fwd2::LAUNCH_REGS)
+        return fail(SA_ERR_UNSUPPORTED, "sparse_fwd2_kernel was built with %d registers per thread, not %d",
+                    fa.numRegs, sa::fwd2::LAUNCH_REGS);
     sa::fwd2::Fwd2Params prm;
     prm.cnt = cnt;
     prm.idx = idx;

@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse attn ms/call & kept-tile TFLOPS vs bf16 peak; speedup vs own dense"
 UNIT = "TFLOP/s (kept tiles)"
 DEFAULT_CONFIG = "wan"
-FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_fwd2_kernel.cuh",
+FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_attn_kernel.cuh",
                "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
 MASK_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
                 "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
@@ -448,7 +448,7 @@ def run_ours(args):
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
                          "traffic": None if tr is None else tr["bytes_per_launch"],
-                         "kernel": "sparse_fwd2_kernel", "peak_source": peaks["source"] + " (burst)",
+                         "kernel": "sparse_attn_fwd_kernel", "peak_source": peaks["source"] + " (burst)",
                          "frac_of_sustained": None if not peaks.get("bf16_tflops_sustained") else
                          fwd_tflops / peaks["bf16_tflops_sustained"]},
             "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": peaks["hbm_gbs"],

@@ -3,7 +3,7 @@
 Method: Cody-Waite style range reduction (x = n + f, n = round(x), f in
 [-1/2, 1/2], 2^x = 2^n * 2^f) and a degree-3 polynomial for 2^f on
 [-1/2, 1/2] chosen by the Remez exchange algorithm to minimise the maximum
-relative error. Run it to print the constants written in sa_fwd2_kernel.cuh.
+relative error. Run it to print the constants written in sa_attn_kernel.cuh.
 """
 import numpy as np
 

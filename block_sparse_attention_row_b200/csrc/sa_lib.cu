@@ -16,7 +16,7 @@
 #include "sparse_attn_testing.h"
 #include "sa_ptx.cuh"
 #include "sa_mask_kernels.cuh"
-#include "sa_fwd2_kernel.cuh"
+#include "sa_attn_kernel.cuh"
 
 namespace {
 
@@ -183,28 +183,41 @@ sa_status launch_select(const Dims& g, const float* in, int ld_in, double k, dou
     return cuda_check(cudaGetLastError(), "select_kernel launch");
 }
 
+// Multiprocessor count of the current device (cached per device).
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <int D, int BQ>
-sa_status launch_fwd2_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
+sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                         const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
                         cudaStream_t st) {
-    using L = sa::fwd2::Layout2<D>;
+    using L = sa::attn::Layout<D>;
     CUtensorMap mq, mk, mv;
     sa_status s;
-    if ((s = make_map(&mq, Q, g, sa::fwd2::MROWS)) != SA_OK) return s;
-    if ((s = make_map(&mk, K, g, sa::fwd2::BK)) != SA_OK) return s;
-    if ((s = make_map(&mv, V, g, sa::fwd2::BK)) != SA_OK) return s;
-    auto kern = sa::fwd2::sparse_fwd2_kernel<D, BQ>;
+    if ((s = make_map(&mq, Q, g, sa::attn::MROWS)) != SA_OK) return s;
+    if ((s = make_map(&mk, K, g, sa::attn::BK)) != SA_OK) return s;
+    if ((s = make_map(&mv, V, g, sa::attn::BK)) != SA_OK) return s;
+    auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ>;
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
-                        "sparse_fwd2_kernel shared-memory attribute")) != SA_OK)
+                        "sparse_attn_fwd_kernel shared-memory attribute")) != SA_OK)
         return s;
     // The kernel moves registers between its warpgroups (setmaxnreg); the
     // split adds up only for the launch register count it was written for.
     cudaFuncAttributes fa;
-    if ((s = cuda_check(cudaFuncGetAttributes(&fa, kern), "sparse_fwd2_kernel attributes")) != SA_OK) return s;
-    if (fa.numRegs != sa::fwd2::LAUNCH_REGS)
-        return fail(SA_ERR_UNSUPPORTED, "sparse_fwd2_kernel was built with %d registers per thread, not %d",
-                    fa.numRegs, sa::fwd2::LAUNCH_REGS);
-    sa::fwd2::Fwd2Params prm;
+    if ((s = cuda_check(cudaFuncGetAttributes(&fa, kern), "sparse_attn_fwd_kernel attributes")) != SA_OK) return s;
+    if (fa.numRegs != sa::attn::LAUNCH_REGS)
+        return fail(SA_ERR_UNSUPPORTED, "sparse_attn_fwd_kernel was built with %d registers per thread, not %d",
+                    fa.numRegs, sa::attn::LAUNCH_REGS);
+    sa::attn::Params prm;
     prm.cnt = cnt;
     prm.idx = idx;
     prm.O = O;
@@ -217,21 +230,23 @@ sa_status launch_fwd2_t(const Dims& g, const void* Q, const void* K, const void*
     prm.out_f32 = out_f32 ? 1 : 0;
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     prm.wait_limit_ns = WAIT_LIMIT_NS;
-    const int grid = (prm.rows + sa::fwd2::NSLOT - 1) / sa::fwd2::NSLOT;
-    kern<<<grid, sa::fwd2::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, prm);
-    return cuda_check(cudaGetLastError(), "sparse_fwd2_kernel launch");
+    // Persistent: one CTA per multiprocessor (fewer when there are fewer row pairs).
+    const int pairs = (prm.rows + sa::attn::NSLOT - 1) / sa::attn::NSLOT;
+    const int grid = pairs < sm_count() ? pairs : sm_count();
+    kern<<<grid, sa::attn::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, prm);
+    return cuda_check(cudaGetLastError(), "sparse_attn_fwd_kernel launch");
 }
 
 sa_status launch_fwd(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                      const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
                      cudaStream_t st) {
     if (g.d == 128 && g.bq == 128)
-        return launch_fwd2_t<128, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<128, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
     if (g.d == 128 && g.bq == 64)
-        return launch_fwd2_t<128, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<128, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
     if (g.d == 64 && g.bq == 128)
-        return launch_fwd2_t<64, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
-    return launch_fwd2_t<64, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<64, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+    return launch_attn_t<64, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
 }
 
 sa_status check_out_dtype(int o_dtype) {
@@ -242,7 +257,7 @@ sa_status check_out_dtype(int o_dtype) {
 
 __global__ void exp2_poly_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) y[i] = sa::fwd2::exp2_poly(x[i]);
+    if (i < n) y[i] = sa::attn::exp2_poly(x[i]);
 }
 
 }  // namespace

@@ -117,7 +117,7 @@ def test_exp2_poly_constants_come_from_the_remez_script():
     spec.loader.exec_module(gen)
     coef, err = gen.remez_relative()
     assert err < 1e-4
-    src = open(os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "sa_fwd2_kernel.cuh")).read()
+    src = open(os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "sa_attn_kernel.cuh")).read()
     body = src[src.index("float exp2_poly("):src.index("return (x == -INFINITY)")]
     lits = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[-+][0-9]+)f", body)]
     assert len(lits) == 4

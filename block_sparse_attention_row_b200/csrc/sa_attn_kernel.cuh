@@ -291,7 +291,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 mbar_init(&B.ch_empty[c], 1);
             }
             mbar_init(&B.s_full, 1);
-            mbar_init(&B.p_full, 128);
+            mbar_init(&B.p_full, 4);   // one arrival per softmax warp
             mbar_init(&B.o_full, 1);
             mbar_init(&B.drain, 1);
         }
@@ -429,7 +429,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 umma_ss_batch<L::SLABS * 4>(tS, ad, bd, IDESC_S, 0u);
             };
             auto wait_chunk = [&](int kk) -> bool {
-                return mbar_wait_bounded(&B.ch_full[kk % NCH], (kk / NCH) & 1, abort_flag, W_CH_FULL, lim);
+                return mbar_wait_spin(&B.ch_full[kk % NCH], (kk / NCH) & 1, abort_flag, W_CH_FULL, lim);
             };
             int k = 0, g = 0, kq = 0, ticket = 0;
             bool ok = true;
@@ -451,9 +451,11 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 ++k;
                 for (int t = 0; t < nt; ++t) {
                     const bool more = t + 1 < nt;
-                    // P_s(t) written (and O_s rescaled), V(t) landed, K(t+1) landed.
-                    if (!mbar_wait_bounded(&B.p_full, g & 1, abort_flag, W_P_FULL, lim) || !wait_chunk(k) ||
-                        (more && !wait_chunk(k + 1))) {
+                    // V(t) landed, K(t+1) landed (both normally long before), and
+                    // P_s(t) written (and O_s rescaled): the batch goes out as soon
+                    // as the softmax hands P over.
+                    if (!wait_chunk(k) || (more && !wait_chunk(k + 1)) ||
+                        !mbar_wait_spin(&B.p_full, g & 1, abort_flag, W_P_FULL, lim)) {
                         ok = false;
                         break;
                     }
@@ -620,7 +622,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&B.p_full);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B.p_full);
                 ++g;
             }
             if (!ok) break;

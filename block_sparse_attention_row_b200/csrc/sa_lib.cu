@@ -170,7 +170,7 @@ sa_status launch_select(const Dims& g, const float* in, int ld_in, double k, dou
                         int32_t* idx, uint8_t* mask, float* P_out, cudaStream_t st) {
     const int rows = g.BH * g.n_q;
     const int wpc = sa::mask::select_warps_per_cta(g.n_k);
-    const size_t smem = (size_t)wpc * 2 * g.n_k * sizeof(uint32_t);
+    const size_t smem = (size_t)wpc * sa::mask::select_row_bytes(g.n_k);
     auto kern = sa::mask::select_kernel<FROM_LOGITS>;
     // Set on every call: the attribute is per device.
     sa_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

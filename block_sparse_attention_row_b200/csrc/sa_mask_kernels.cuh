@@ -84,16 +84,19 @@ pool_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
 }
 
 // logits[bh*n_q + i][j] = scale * sum_c Qbar[bh,i,c] * Kbar[bh,j,c], fp32.
-// CTA tile: 32 query blocks x 64 key blocks, channels in chunks of 64; each
-// thread accumulates 2 x 4 outputs.
-constexpr int SC_TI = 32, SC_TJ = 64, SC_TC = 64, SC_THREADS = 256;
+// CTA tile: 64 query blocks x 128 key blocks, channels in chunks of 32 held
+// channel-major in shared memory; each of the 256 threads accumulates 4 query
+// blocks x 8 key blocks (two groups of 4 adjacent key blocks, 64 apart), so
+// one channel step is 32 FMAs for three 16-byte shared-memory loads.
+constexpr int SC_TI = 64, SC_TJ = 128, SC_TC = 32, SC_THREADS = 256;
 
 template <int D>
 __global__ void __launch_bounds__(SC_THREADS)
 score_kernel(const float* __restrict__ Qbar, const float* __restrict__ Kbar,
              float* __restrict__ logits, int ld, int n_q, int n_k, float scale) {
-    __shared__ __align__(16) float qs[SC_TI][SC_TC + 4];
-    __shared__ __align__(16) float kt[SC_TC][SC_TJ];
+    static_assert(D % SC_TC == 0, "channel chunks");
+    __shared__ __align__(16) float qs[SC_TC][SC_TI];
+    __shared__ __align__(16) float ks[SC_TC][SC_TJ];
 
     const int bh = blockIdx.z;
     const int i0 = blockIdx.y * SC_TI;
@@ -101,65 +104,65 @@ score_kernel(const float* __restrict__ Qbar, const float* __restrict__ Kbar,
     const int t = threadIdx.x;
     const float* qsrc = Qbar + (size_t)bh * n_q * D;
     const float* ksrc = Kbar + (size_t)bh * n_k * D;
-    const int tr = t / 16, tj = t % 16;
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int ty = t / 16, tx = t % 16;   // rows 4ty..4ty+3; keys 4tx..4tx+3 and 64+4tx..64+4tx+3
+    float acc[4][8];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
 
     for (int c0 = 0; c0 < D; c0 += SC_TC) {
-        // Q tile, row-major (float4 along channels, coalesced).
+        // Tiles transposed to [channel][row]. Consecutive threads take
+        // consecutive rows, so the transposed shared-memory stores are free of
+        // bank conflicts (the 16-byte global reads are then 512 bytes apart).
         for (int e = t; e < SC_TI * (SC_TC / 4); e += SC_THREADS) {
-            const int r = e / (SC_TC / 4), c4 = e % (SC_TC / 4);
+            const int r = e % SC_TI, c4 = e / SC_TI;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i0 + r < n_q)
-                v = *reinterpret_cast<const float4*>(qsrc + (size_t)(i0 + r) * D + c0 + 4 * c4);
-            *reinterpret_cast<float4*>(&qs[r][4 * c4]) = v;
+            if (i0 + r < n_q) v = *reinterpret_cast<const float4*>(qsrc + (size_t)(i0 + r) * D + c0 + 4 * c4);
+            qs[4 * c4 + 0][r] = v.x;
+            qs[4 * c4 + 1][r] = v.y;
+            qs[4 * c4 + 2][r] = v.z;
+            qs[4 * c4 + 3][r] = v.w;
         }
-        // K tile, transposed to [channel][key] so that consecutive threads
-        // read consecutive keys below.
         for (int e = t; e < SC_TJ * (SC_TC / 4); e += SC_THREADS) {
-            const int j = e % SC_TJ, c4 = e / SC_TJ;
+            const int jj = e % SC_TJ, c4 = e / SC_TJ;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (j0 + j < n_k)
-                v = *reinterpret_cast<const float4*>(ksrc + (size_t)(j0 + j) * D + c0 + 4 * c4);
-            kt[4 * c4 + 0][j] = v.x;
-            kt[4 * c4 + 1][j] = v.y;
-            kt[4 * c4 + 2][j] = v.z;
-            kt[4 * c4 + 3][j] = v.w;
+            if (j0 + jj < n_k) v = *reinterpret_cast<const float4*>(ksrc + (size_t)(j0 + jj) * D + c0 + 4 * c4);
+            ks[4 * c4 + 0][jj] = v.x;
+            ks[4 * c4 + 1][jj] = v.y;
+            ks[4 * c4 + 2][jj] = v.z;
+            ks[4 * c4 + 3][jj] = v.w;
         }
         __syncthreads();
-#pragma unroll 4
-        for (int c = 0; c < SC_TC; c += 4) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&qs[2 * tr][c]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&qs[2 * tr + 1][c]);
-            const float q0v[4] = {q0.x, q0.y, q0.z, q0.w};
-            const float q1v[4] = {q1.x, q1.y, q1.z, q1.w};
+#pragma unroll 8
+        for (int c = 0; c < SC_TC; ++c) {
+            const float4 a = *reinterpret_cast<const float4*>(&qs[c][4 * ty]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&ks[c][4 * tx]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&ks[c][64 + 4 * tx]);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const float4 kv = *reinterpret_cast<const float4*>(&kt[c + cc][4 * tj]);
-                a0[0] = fmaf(q0v[cc], kv.x, a0[0]);
-                a0[1] = fmaf(q0v[cc], kv.y, a0[1]);
-                a0[2] = fmaf(q0v[cc], kv.z, a0[2]);
-                a0[3] = fmaf(q0v[cc], kv.w, a0[3]);
-                a1[0] = fmaf(q1v[cc], kv.x, a1[0]);
-                a1[1] = fmaf(q1v[cc], kv.y, a1[1]);
-                a1[2] = fmaf(q1v[cc], kv.z, a1[2]);
-                a1[3] = fmaf(q1v[cc], kv.w, a1[3]);
-            }
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[r][q] = fmaf(av[r], bv[q], acc[r][q]);
         }
         __syncthreads();
     }
-    const int jj = j0 + 4 * tj;
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const int i = i0 + 2 * tr + rr;
+    for (int r = 0; r < 4; ++r) {
+        const int i = i0 + 4 * ty + r;
         if (i >= n_q) continue;
-        const float* a = rr ? a1 : a0;
-        float* dst = logits + ((size_t)bh * n_q + i) * ld + jj;
-        if (jj + 3 < ld) {
-            *reinterpret_cast<float4*>(dst) =
-                make_float4(a[0] * scale, a[1] * scale, a[2] * scale, a[3] * scale);
-        } else {
-            for (int e = 0; e < 4; ++e)
-                if (jj + e < ld) dst[e] = a[e] * scale;
+        float* row = logits + ((size_t)bh * n_q + i) * ld;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const int jj = j0 + 64 * g + 4 * tx;
+            const float* a = &acc[r][4 * g];
+            if (jj + 3 < ld) {
+                *reinterpret_cast<float4*>(row + jj) = make_float4(a[0] * scale, a[1] * scale, a[2] * scale, a[3] * scale);
+            } else {
+                for (int e = 0; e < 4; ++e)
+                    if (jj + e < ld) row[jj + e] = a[e] * scale;
+            }
         }
     }
 }
@@ -187,12 +190,14 @@ __device__ __forceinline__ uint64_t fixed_mass(uint32_t bits) {
 // unsigned order is numeric order). For the metric "fixed-point mass"
 // (MASS = true) or "number of entries" (MASS = false) it finds the largest
 // 31-bit value v such that the metric summed over the entries >= v still
-// reaches `target`, most significant bit first. The entries still able to
-// decide the answer (those inside the current range [v, v | (2^(b+1) - 1)])
-// are kept in `work` and compacted in place after every bit, so each step
-// only touches the survivors. Returns v and, through the out-parameters, the
-// count and mass of the entries strictly above v. Integer sums only: the
-// answer does not depend on the order of the reductions.
+// reaches `target`, most significant bit first. After bit b is decided, the
+// entries still able to decide the answer are those that agree with v on the
+// bits above b; while there are more than 32 of them each step rescans the row
+// and tests that prefix, and once at most 32 are left they are gathered into
+// one register per lane and the remaining bits take one ballot each. Returns
+// v and, through the out-parameters, the count and mass of the entries
+// strictly above v. Integer sums only: the answer does not depend on the
+// order of the reductions.
 struct Boundary {
     uint32_t v;
     int n_above;
@@ -200,54 +205,77 @@ struct Boundary {
 };
 
 template <bool MASS>
-__device__ Boundary boundary_search(const uint32_t* __restrict__ bits, uint32_t* __restrict__ work,
+__device__ Boundary boundary_search(const uint32_t* __restrict__ bits, const uint64_t* __restrict__ masses,
                                     int n, uint64_t target, int lane) {
-    for (int j = lane; j < n; j += 32) work[j] = bits[j];
-    __syncwarp();
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    int m = n;
     uint32_t v = 0;
     int n_above = 0;
     uint64_t mass_above = 0;
-    for (int b = 30; b >= 0; --b) {
+    int m = n;    // entries that agree with v on the bits decided so far
+    int b = 30;   // bit 31 is the sign, 0 for every score
+    for (; b >= 0 && m > 32; --b) {
         const uint32_t bit = 1u << b;
-        uint64_t hi_mass = 0;
         uint32_t hi_cnt = 0;
-        for (int j = lane; j < m; j += 32) {
-            const uint32_t x = work[j];
-            if (x & bit) {
+        uint64_t hi_mass = 0;
+        for (int j = lane; j < n; j += 32) {
+            const uint32_t x = bits[j];
+            if ((((x ^ v) >> b) >> 1) == 0u && (x & bit)) {
                 ++hi_cnt;
-                if (MASS) hi_mass += fixed_mass(x);
+                if (MASS) hi_mass += masses[j];
             }
         }
         hi_cnt = warp_sum_u32(hi_cnt);
         if (MASS) hi_mass = warp_sum_u64(hi_mass);
         const uint64_t reach = MASS ? mass_above + hi_mass : (uint64_t)(n_above + (int)hi_cnt);
-        const bool take = reach >= target;
-        if (take) {
+        if (reach >= target) {
             v |= bit;  // entries without this bit fall below v
+            m = (int)hi_cnt;
         } else {
             n_above += (int)hi_cnt;  // entries with this bit lie above the range
             mass_above += hi_mass;
+            m -= (int)hi_cnt;
         }
-        const int keep_n = take ? (int)hi_cnt : m - (int)hi_cnt;
-        if (keep_n != m) {
-            int out = 0;
-            for (int base = 0; base < m; base += 32) {
-                const int j = base + lane;
-                uint32_t x = 0;
-                bool keep = false;
-                if (j < m) {
-                    x = work[j];
-                    keep = ((x & bit) != 0) == take;
+    }
+    if (b >= 0) {
+        // At most 32 candidates left: one per lane.
+        uint32_t x = 0;
+        uint64_t xm = 0;
+        int got = 0;
+        for (int base = 0; base < n; base += 32) {
+            const int j = base + lane;
+            const bool cand = j < n && ((((bits[j] ^ v) >> b) >> 1) == 0u);
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, cand);
+            const uint32_t xj = cand ? bits[j] : 0u;
+            const uint64_t mj = (MASS && cand) ? masses[j] : 0ull;
+            // Hand candidate number `slot` to lane `slot`.
+#pragma unroll 1
+            for (uint32_t rest = bal; rest; rest &= rest - 1) {
+                const int src = __ffs(rest) - 1;
+                const int dst = got + __popc(bal & ((1u << src) - 1u));
+                const uint32_t xv = __shfl_sync(0xFFFFFFFFu, xj, src);
+                const uint64_t mv = MASS ? __shfl_sync(0xFFFFFFFFu, mj, src) : 0ull;
+                if (lane == dst) {
+                    x = xv;
+                    xm = mv;
                 }
-                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, keep);
-                __syncwarp();
-                if (keep) work[out + __popc(bal & lt_mask)] = x;
-                out += __popc(bal);
-                __syncwarp();
             }
-            m = keep_n;
+            got += __popc(bal);
+        }
+        bool alive = lane < got;
+        for (; b >= 0; --b) {
+            const uint32_t bit = 1u << b;
+            const bool hi = alive && (x & bit);
+            const uint32_t hi_bal = __ballot_sync(0xFFFFFFFFu, hi);
+            const uint32_t hi_cnt = __popc(hi_bal);
+            const uint64_t hi_mass = MASS ? warp_sum_u64(hi ? xm : 0ull) : 0ull;
+            const uint64_t reach = MASS ? mass_above + hi_mass : (uint64_t)(n_above + (int)hi_cnt);
+            if (reach >= target) {
+                v |= bit;
+                alive = hi;
+            } else {
+                n_above += (int)hi_cnt;
+                mass_above += hi_mass;
+                alive = alive && !(x & bit);
+            }
         }
     }
     if (!MASS) mass_above = 0;
@@ -258,9 +286,11 @@ constexpr int SEL_MAX_WARPS = 4;
 constexpr int SEL_SMEM_BUDGET = 200 * 1024;
 
 // Warps (rows) per CTA of select_kernel for a row length n_k: each warp
-// holds its row twice in shared memory (8 bytes per entry).
+// holds its row's score bits and fixed-point masses in shared memory (12
+// bytes per entry, rounded up to keep the masses 8-byte aligned).
+__host__ __device__ inline int select_row_bytes(int n_k) { return 4 * ((n_k + 1) & ~1) + 8 * n_k; }
 inline int select_warps_per_cta(int n_k) {
-    int w = SEL_SMEM_BUDGET / (8 * n_k);
+    int w = SEL_SMEM_BUDGET / select_row_bytes(n_k);
     return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : w);
 }
 
@@ -278,13 +308,13 @@ __global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
 select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
               int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
               float* __restrict__ P_out) {
-    extern __shared__ uint32_t sel_smem[];
+    extern __shared__ __align__(8) unsigned char sel_smem[];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int wpc = blockDim.x / 32;
     const long long row = (long long)blockIdx.x * wpc + warp;
     if (row >= n_rows) return;
-    uint32_t* bits = sel_smem + (size_t)warp * 2 * n_k;
-    uint32_t* work = bits + n_k;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(sel_smem + (size_t)warp * select_row_bytes(n_k));
+    uint64_t* masses = reinterpret_cast<uint64_t*>(bits + ((n_k + 1) & ~1));
     const float* src = in + (size_t)row * ld_in;
 
     if (FROM_LOGITS) {
@@ -292,16 +322,21 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
         for (int j = lane; j < n_k; j += 32) mx = fmaxf(mx, src[j]);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        // exp(x - max) as 2^((x - max) log2 e) on the MUFU unit (relative error
+        // about 2e-7, far below the 1e-6 near-tie scale), and one reciprocal of
+        // the sum; P is clamped to 1 so its fixed-point mass stays <= 2^31.
+        const float mxl = mx * 1.4426950408889634f;
         float sum = 0.f;
         for (int j = lane; j < n_k; j += 32) {
-            const float e = expf(src[j] - mx);
+            const float e = ex2_approx(fmaf(src[j], 1.4426950408889634f, -mxl));
             bits[j] = __float_as_uint(e);
             sum += e;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        const float inv = 1.0f / sum;
         for (int j = lane; j < n_k; j += 32) {
-            const float pj = __fdiv_rn(__uint_as_float(bits[j]), sum);
+            const float pj = fminf(__uint_as_float(bits[j]) * inv, 1.0f);
             bits[j] = __float_as_uint(pj);
             if (P_out) P_out[(size_t)row * n_k + j] = pj;
         }
@@ -324,13 +359,18 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
     Boundary bd = {0u, 0, 0ull};
     if (p >= 1.0) {
         L = n_k;
-    } else {
+    } else if (p > 0.0) {
         uint64_t w = 0;
-        for (int j = lane; j < n_k; j += 32) w += fixed_mass(bits[j]);
+        for (int j = lane; j < n_k; j += 32) {
+            const uint64_t mj = fixed_mass(bits[j]);
+            masses[j] = mj;
+            w += mj;
+        }
         const uint64_t W = warp_sum_u64(w);
         const uint64_t T = (uint64_t)ceil(p * (double)W);
+        __syncwarp();
         if (T > 0) {
-            const Boundary mb = boundary_search<true>(bits, work, n_k, T, lane);
+            const Boundary mb = boundary_search<true>(bits, masses, n_k, T, lane);
             const uint64_t wb = fixed_mass(mb.v);  // > 0 for scores in [0, 1]
             const uint64_t need = wb ? (T - mb.mass_above + wb - 1) / wb : 1;
             const int m_p = (int)(mb.n_above + need);
@@ -355,7 +395,7 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
         if (mask_row)
             for (int j = lane; j < n_k; j += 32) mask_row[j] = 0;
     } else {
-        if (!have_boundary) bd = boundary_search<false>(bits, work, n_k, (uint64_t)L, lane);
+        if (!have_boundary) bd = boundary_search<false>(bits, masses, n_k, (uint64_t)L, lane);
         const uint32_t v = bd.v;
         const int ties_kept = L - bd.n_above;
         int ties_before = 0, kept_before = 0;

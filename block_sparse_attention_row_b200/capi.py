@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 # Every entry point declared in include/sparse_attn.h and include/sparse_attn_testing.h.
 EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_mask_noalloc",
             "sparse_attn_select",
-            "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_check_device_error",
+            "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
+            "sparse_attn_host", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_exp2_poly")
 
 
@@ -72,6 +73,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_fwd.restype = ctypes.c_int
         lib.sparse_attn_fwd_dense.argtypes = [sp, vp, vp, vp, vp, ctypes.c_int, f32p, vp]
         lib.sparse_attn_fwd_dense.restype = ctypes.c_int
+        lib.sparse_attn_host_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
+        lib.sparse_attn_host_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_host.argtypes = [sp, vp, vp, vp, ctypes.c_double, ctypes.c_double, vp, ctypes.c_int,
+                                         i32p, i32p, ctypes.c_int, vp, ctypes.c_size_t, vp]
+        lib.sparse_attn_host.restype = ctypes.c_int
         lib.sparse_attn_check_device_error.argtypes = [vp]
         lib.sparse_attn_check_device_error.restype = ctypes.c_int
         lib.sparse_attn_last_error.argtypes = []
@@ -262,6 +268,59 @@ def sparse_attn(Q, K, V, bq: int, bk: int, k: float, p: float, *, stream=None):
     m = sparse_attn_mask(Q, K, bq, bk, k, p, stream=stream)
     O = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, bk, stream=stream)
     return O, m["cnt"], m["idx"]
+
+
+def host_workspace_bytes(B: int, H: int, N: int, d: int, bq: int, bk: int,
+                         out_dtype=torch.bfloat16, heads_per_chunk: int = 0) -> int:
+    od = SA_F32 if out_dtype == torch.float32 else SA_BF16
+    sh = make_shape(B, H, N, d, bq, bk)
+    n = load_library().sparse_attn_host_workspace_bytes(ctypes.byref(sh), od, int(heads_per_chunk))
+    if n == 0:
+        raise ValueError("unsupported shape, output type or heads_per_chunk")
+    return int(n)
+
+
+def sparse_attn_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bq: int, bk: int, k: float, p: float,
+                     *, device=None, out_dtype=torch.bfloat16, want_cnt: bool = False, want_idx: bool = False,
+                     heads_per_chunk: int = 0, out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> dict:
+    """The whole path on host tensors (page-locked for overlap): copies, mask and
+    attention pipelined by chunks of heads on the library's streams.
+
+    Returns host tensors {"O", and "cnt"/"idx" if requested}; they are ready
+    once `stream` (default: the device's current stream) has reached this call.
+    """
+    for t in (Q, K, V):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("Q, K, V must be contiguous bf16 host tensors of shape [B, H, N, d]")
+        if t.shape != Q.shape:
+            raise ValueError("Q, K, V must share shape")
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if dev.type != "cuda":
+        raise ValueError("device must be a CUDA device")
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    od = SA_F32 if out_dtype == torch.float32 else SA_BF16
+    pin = Q.is_pinned()
+    out = {} if out is None else out
+    if "O" not in out:
+        out["O"] = torch.empty(B, H, N, d, dtype=out_dtype, pin_memory=pin)
+    if want_cnt and "cnt" not in out:
+        out["cnt"] = torch.empty(B, H, n_q, dtype=torch.int32, pin_memory=pin)
+    if want_idx and "idx" not in out:
+        out["idx"] = torch.empty(B, H, n_q, n_k, dtype=torch.int32, pin_memory=pin)
+    need = host_workspace_bytes(B, H, N, d, bq, bk, out_dtype, heads_per_chunk)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    sh = make_shape(B, H, N, d, bq, bk)
+    st = load_library().sparse_attn_host(
+        ctypes.byref(sh), _ptr(Q), _ptr(K), _ptr(V), float(k), float(p), _ptr(out["O"]), od,
+        _ptr(out.get("cnt") if want_cnt else None), _ptr(out.get("idx") if want_idx else None),
+        int(heads_per_chunk), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(dev, stream))
+    _check("sparse_attn_host", st)
+    out["workspace"] = workspace
+    return out
 
 
 def check_device_error(device=None, stream=None) -> None:

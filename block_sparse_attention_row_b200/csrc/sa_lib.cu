@@ -428,6 +428,192 @@ sa_status sparse_attn_check_device_error(void* stream) {
                 rec.info, rec.block, rec.thread);
 }
 
+// ------------------------------------------------- host-buffer pipeline
+}  // extern "C"
+
+namespace {
+
+// Chunk geometry and device-buffer layout of sparse_attn_host.
+struct HostPlan {
+    Dims g;
+    int hpc;             // heads per chunk
+    int nchunk;
+    size_t esize_o;      // bytes per O element
+    size_t qkv_bytes;    // one chunk of Q (or K, or V)
+    size_t o_bytes, cnt_bytes, idx_bytes, mws_bytes;
+    size_t off_q[2], off_k[2], off_v[2], off_o[2], off_cnt[2], off_idx[2], off_mws[2];
+    size_t total;
+};
+
+constexpr int HOST_MIN_ROWS_PER_CHUNK = 2368;   // ~8 query-block rows per attention pipeline on 148 SMs
+
+sa_status host_plan(const sa_shape* shape, int o_dtype, int heads_per_chunk, HostPlan& hp) {
+    sa_status s;
+    if ((s = check_shape(shape, hp.g)) != SA_OK) return s;
+    if ((s = check_out_dtype(o_dtype)) != SA_OK) return s;
+    if (heads_per_chunk < 0) return fail(SA_ERR_INVALID_ARG, "heads_per_chunk=%d", heads_per_chunk);
+    const Dims& g = hp.g;
+    int hpc = heads_per_chunk;
+    if (hpc == 0) hpc = (HOST_MIN_ROWS_PER_CHUNK + g.n_q - 1) / g.n_q;
+    if (hpc > g.BH) hpc = g.BH;
+    hp.hpc = hpc;
+    hp.nchunk = (g.BH + hpc - 1) / hpc;
+    hp.esize_o = (o_dtype == SA_F32) ? 4 : 2;
+    const size_t tok = (size_t)hpc * g.N * g.d;
+    hp.qkv_bytes = tok * 2;
+    hp.o_bytes = tok * hp.esize_o;
+    hp.cnt_bytes = (size_t)hpc * g.n_q * 4;
+    hp.idx_bytes = (size_t)hpc * g.n_q * g.n_k * 4;
+    Dims sub = g;
+    sub.B = 1;
+    sub.H = hpc;
+    sub.BH = hpc;
+    hp.mws_bytes = workspace_layout(sub).total;
+    size_t off = 0;
+    for (int b = 0; b < 2; ++b) {
+        hp.off_q[b] = off; off += round256(hp.qkv_bytes);
+        hp.off_k[b] = off; off += round256(hp.qkv_bytes);
+        hp.off_v[b] = off; off += round256(hp.qkv_bytes);
+        hp.off_o[b] = off; off += round256(hp.o_bytes);
+        hp.off_cnt[b] = off; off += round256(hp.cnt_bytes);
+        hp.off_idx[b] = off; off += round256(hp.idx_bytes);
+        hp.off_mws[b] = off; off += round256(hp.mws_bytes);
+    }
+    hp.total = off;
+    return SA_OK;
+}
+
+// The library's three streams on the current device (copy-in, compute,
+// copy-out), created on first use and kept for the life of the process.
+sa_status host_streams(cudaStream_t (&out)[3]) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][3] = {};
+    int dev = 0;
+    sa_status s;
+    if ((s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) != SA_OK) return s;
+    if (dev < 0 || dev >= 64) return fail(SA_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 3; ++i) {
+        if (!streams[dev][i] &&
+            (s = cuda_check(cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking),
+                            "create a pipeline stream")) != SA_OK)
+            return s;
+        out[i] = streams[dev][i];
+    }
+    return SA_OK;
+}
+
+// Events of one call, destroyed when the call returns (a destroyed event
+// that is still pending completes normally).
+struct CallEvents {
+    cudaEvent_t ev[7] = {};
+    ~CallEvents() {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+    }
+    sa_status create() {
+        for (cudaEvent_t& e : ev) {
+            sa_status s = cuda_check(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "create an event");
+            if (s != SA_OK) return s;
+        }
+        return SA_OK;
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+size_t sparse_attn_host_workspace_bytes(const sa_shape* shape, int o_dtype, int heads_per_chunk) {
+    HostPlan hp;
+    if (host_plan(shape, o_dtype, heads_per_chunk, hp) != SA_OK) return 0;
+    return hp.total;
+}
+
+sa_status sparse_attn_host(const sa_shape* shape, const void* Q, const void* K, const void* V, double k,
+                           double p, void* O, int o_dtype, int32_t* cnt_or_null, int32_t* idx_or_null,
+                           int heads_per_chunk, void* workspace, size_t workspace_bytes, void* stream) {
+    HostPlan hp;
+    sa_status s;
+    if ((s = host_plan(shape, o_dtype, heads_per_chunk, hp)) != SA_OK) return s;
+    if ((s = check_kp(k, p)) != SA_OK) return s;
+    if (!Q || !K || !V || !O || !workspace)
+        return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, O, workspace");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+        (cnt_or_null && !aligned16(cnt_or_null)) || (idx_or_null && !aligned16(idx_or_null)) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required; 256 for workspace)");
+    if (workspace_bytes < hp.total)
+        return fail(SA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, hp.total);
+    cudaStream_t ps[3];
+    if ((s = host_streams(ps)) != SA_OK) return s;
+    const cudaStream_t s_in = ps[0], s_comp = ps[1], s_out = ps[2];
+    const cudaStream_t caller = reinterpret_cast<cudaStream_t>(stream);
+    CallEvents E;
+    if ((s = E.create()) != SA_OK) return s;
+    cudaEvent_t ev_start = E.ev[0], ev_in[2] = {E.ev[1], E.ev[2]}, ev_comp[2] = {E.ev[3], E.ev[4]},
+                ev_out[2] = {E.ev[5], E.ev[6]};
+    const Dims& g = hp.g;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    // Start after the caller's stream.
+    if ((s = cuda_check(cudaEventRecord(ev_start, caller), "record the start event")) != SA_OK) return s;
+    for (cudaStream_t st : ps)
+        if ((s = cuda_check(cudaStreamWaitEvent(st, ev_start, 0), "order after the caller's stream")) != SA_OK)
+            return s;
+    const size_t tok_bytes = (size_t)g.N * g.d * 2;   // one head of Q, K or V
+    for (int c = 0; c < hp.nchunk; ++c) {
+        const int b = c & 1;
+        const int bh0 = c * hp.hpc;
+        const int hc = (g.BH - bh0 < hp.hpc) ? g.BH - bh0 : hp.hpc;
+        const sa_shape sub = {1, hc, g.N, g.d, g.bq, g.bk};
+        void* Qd = ws + hp.off_q[b];
+        void* Kd = ws + hp.off_k[b];
+        void* Vd = ws + hp.off_v[b];
+        void* Od = ws + hp.off_o[b];
+        int32_t* cntd = reinterpret_cast<int32_t*>(ws + hp.off_cnt[b]);
+        int32_t* idxd = reinterpret_cast<int32_t*>(ws + hp.off_idx[b]);
+        const size_t in_bytes = (size_t)hc * tok_bytes;
+        // Copy in, once the compute of chunk c-2 no longer reads buffer b.
+        if (c >= 2 && (s = cuda_check(cudaStreamWaitEvent(s_in, ev_comp[b], 0), "order copy-in")) != SA_OK) return s;
+        if ((s = cuda_check(cudaMemcpyAsync(Qd, static_cast<const uint8_t*>(Q) + (size_t)bh0 * tok_bytes, in_bytes,
+                                            cudaMemcpyHostToDevice, s_in), "copy Q in")) != SA_OK ||
+            (s = cuda_check(cudaMemcpyAsync(Kd, static_cast<const uint8_t*>(K) + (size_t)bh0 * tok_bytes, in_bytes,
+                                            cudaMemcpyHostToDevice, s_in), "copy K in")) != SA_OK ||
+            (s = cuda_check(cudaMemcpyAsync(Vd, static_cast<const uint8_t*>(V) + (size_t)bh0 * tok_bytes, in_bytes,
+                                            cudaMemcpyHostToDevice, s_in), "copy V in")) != SA_OK ||
+            (s = cuda_check(cudaEventRecord(ev_in[b], s_in), "record copy-in")) != SA_OK)
+            return s;
+        // Compute, once chunk c is in and the copy-out of chunk c-2 has read buffer b.
+        if ((s = cuda_check(cudaStreamWaitEvent(s_comp, ev_in[b], 0), "order compute")) != SA_OK) return s;
+        if (c >= 2 && (s = cuda_check(cudaStreamWaitEvent(s_comp, ev_out[b], 0), "order compute")) != SA_OK) return s;
+        if ((s = sparse_attn_mask(&sub, Qd, Kd, k, p, cntd, idxd, nullptr, nullptr, ws + hp.off_mws[b], s_comp)) != SA_OK)
+            return s;
+        if ((s = sparse_attn_fwd(&sub, Qd, Kd, Vd, cntd, idxd, Od, o_dtype, nullptr, s_comp)) != SA_OK) return s;
+        if ((s = cuda_check(cudaEventRecord(ev_comp[b], s_comp), "record compute")) != SA_OK) return s;
+        // Copy out.
+        if ((s = cuda_check(cudaStreamWaitEvent(s_out, ev_comp[b], 0), "order copy-out")) != SA_OK) return s;
+        if ((s = cuda_check(cudaMemcpyAsync(static_cast<uint8_t*>(O) + (size_t)bh0 * g.N * g.d * hp.esize_o, Od,
+                                            (size_t)hc * g.N * g.d * hp.esize_o, cudaMemcpyDeviceToHost, s_out),
+                            "copy O out")) != SA_OK)
+            return s;
+        if (cnt_or_null &&
+            (s = cuda_check(cudaMemcpyAsync(cnt_or_null + (size_t)bh0 * g.n_q, cntd, (size_t)hc * g.n_q * 4,
+                                            cudaMemcpyDeviceToHost, s_out), "copy cnt out")) != SA_OK)
+            return s;
+        if (idx_or_null &&
+            (s = cuda_check(cudaMemcpyAsync(idx_or_null + (size_t)bh0 * g.n_q * g.n_k, idxd,
+                                            (size_t)hc * g.n_q * g.n_k * 4, cudaMemcpyDeviceToHost, s_out),
+                            "copy idx out")) != SA_OK)
+            return s;
+        if ((s = cuda_check(cudaEventRecord(ev_out[b], s_out), "record copy-out")) != SA_OK) return s;
+    }
+    // The caller's stream waits for the last copy-out (the copy-out stream is
+    // in order, and it waited for every compute, which waited for every copy-in).
+    if ((s = cuda_check(cudaStreamWaitEvent(caller, ev_out[(hp.nchunk - 1) & 1], 0), "order the caller's stream")) != SA_OK)
+        return s;
+    return ok();
+}
+
 const char* sparse_attn_last_error(void) { return t_last_error.c_str(); }
 
 const char* sparse_attn_version(void) { return "sparse_attn 0.1 (sm_100a)"; }

@@ -30,7 +30,8 @@
  *   where n_q = ceil(N / bq) and n_k = ceil(N / bk).
  * - Every pointer argument is a DEVICE pointer unless stated otherwise; the
  *   caller allocates and owns every buffer. The library allocates no memory
- *   per call; it keeps one small device error record per loaded module.
+ *   per call; it keeps one small device error record per loaded module (and,
+ *   once sparse_attn_host has run on a device, three streams there).
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream). Calls only enqueue work; results are ready when the stream is.
  * - Supported shapes: d in {64, 128}; bq in {64, 128}; bk = 64;
@@ -153,6 +154,42 @@ sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, c
 sa_status sparse_attn_fwd_dense(const sa_shape* shape, const void* Q, const void* K,
                                 const void* V, void* O, int o_dtype, float* lse_or_null,
                                 void* stream);
+
+/* Bytes of device workspace sparse_attn_host needs for `shape` with chunks of
+ * `heads_per_chunk` (b, h) heads (0 = the library's choice, see below): two
+ * device copies of a chunk of Q, K, V and O (O in the element type o_dtype),
+ * of its cnt and idx, and of the mask workspace of a chunk. 0 on an invalid
+ * shape, o_dtype or heads_per_chunk. */
+size_t sparse_attn_host_workspace_bytes(const sa_shape* shape, int o_dtype, int heads_per_chunk);
+
+/* The whole path (steps 1-4: sparse_attn_mask, then sparse_attn_fwd) on HOST
+ * buffers. It has no counterpart in the papers: it packages the same
+ * computation for callers whose Q, K, V are in host memory, overlapping the
+ * PCIe copies with the GPU work. The (b, h) heads are independent rows of the
+ * mask and of the attention, so they are processed in chunks of
+ * heads_per_chunk heads (0 = enough heads for at least 2,368 query-block rows
+ * per chunk, about 8 rows per attention pipeline of a B200): while chunk c is
+ * computed, chunk c+1 is copied to the device and chunk c-1's results back to
+ * the host, on three streams owned by the library, with two device copies of
+ * every chunk buffer (in `workspace`). The results are those of the device
+ * entry points on the whole tensors, bit for bit.
+ * Host pointers: Q, K, V bf16 [B,H,N,d]; O [B,H,N,d] of type o_dtype; cnt
+ *          int32 [B,H,n_q] and idx int32 [B,H,n_q,n_k] (each may be NULL: not
+ *          copied back). They must be page-locked (cudaHostAlloc or
+ *          cudaHostRegister) for the copies to run asynchronously; pageable
+ *          memory works but each copy then blocks the host. 16-byte aligned.
+ * workspace: device, sparse_attn_host_workspace_bytes(shape, o_dtype,
+ *          heads_per_chunk) bytes, 256-byte aligned; workspace_bytes is
+ *          checked against that size.
+ * Ordering: the call's work starts after the work already in `stream` and
+ *          `stream` waits for all of it; host buffers may be read or written
+ *          by the host only once `stream` has reached that point. An error
+ *          returned after the first chunk was enqueued leaves earlier chunks'
+ *          copies in flight (they finish on their own). */
+sa_status sparse_attn_host(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                           double k, double p, void* O, int o_dtype,
+                           int32_t* cnt_or_null, int32_t* idx_or_null, int heads_per_chunk,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (SA_OK if none) and clears the record. */

@@ -124,3 +124,37 @@ def test_exp2_poly_constants_come_from_the_remez_script():
     c3, c2, c1, c0 = lits
     import numpy as np
     assert np.allclose([c0, c1, c2, c3], np.float32(coef), rtol=0, atol=2e-9)
+
+
+def test_host_pipeline_workspace_and_validation(lib):
+    """sparse_attn_host: chunk planning and host-side argument checks (nothing enqueued)."""
+    from block_sparse_attention_row_b200.capi import host_workspace_bytes, make_shape
+    r = lambda x: (x + 255) // 256 * 256
+    B, H, N, d = 1, 40, 32760, 128
+    n_q, n_k = -(-N // 128), -(-N // 64)
+    for hpc, out_dtype, esize in ((0, 0, 2), (3, 0, 2), (7, 1, 4), (40, 0, 2), (100, 0, 2)):
+        got = lib.sparse_attn_host_workspace_bytes(ctypes.byref(make_shape(B, H, N, d, 128, 64)), out_dtype, hpc)
+        h = min(H, -(-2368 // n_q)) if hpc == 0 else min(hpc, H)
+        ld = (n_k + 3) // 4 * 4
+        mws = r(h * n_q * d * 4) + r(h * n_k * d * 4) + r(h * n_q * ld * 4)
+        per = 3 * r(h * N * d * 2) + r(h * N * d * esize) + r(h * n_q * 4) + r(h * n_q * n_k * 4) + r(mws)
+        assert got == 2 * per, (hpc, got, 2 * per)
+    good = ctypes.byref(make_shape(1, 2, 4096, 64, 64, 64))
+    assert lib.sparse_attn_host_workspace_bytes(good, 0, -1) == 0
+    assert lib.sparse_attn_host_workspace_bytes(good, 9, 0) == 0
+    a = ctypes.c_void_p(16)
+    z = ctypes.c_void_p(0)
+    need = lib.sparse_attn_host_workspace_bytes(good, 0, 0)
+    ws = ctypes.c_void_p(256)
+    assert lib.sparse_attn_host(good, a, a, a, 0.1, 0.9, a, 0, None, None, 0, ws, need - 1, None) == 1
+    assert b"workspace" in _host_msg(lib)
+    assert lib.sparse_attn_host(good, z, a, a, 0.1, 0.9, a, 0, None, None, 0, ws, need, None) == 1
+    assert lib.sparse_attn_host(good, a, a, a, 0.0, 0.0, a, 0, None, None, 0, ws, need, None) == 1
+    assert lib.sparse_attn_host(good, a, a, a, 0.1, 0.9, a, 0, None, None, 0, ctypes.c_void_p(16), need, None) == 1
+    assert lib.sparse_attn_host(good, a, a, a, 0.1, 0.9, a, 5, None, None, 0, ws, need, None) == 1
+    assert lib.sparse_attn_host(good, a, a, a, 0.1, 0.9, a, 0, None, None, -2, ws, need, None) == 1
+    assert _host_msg(lib).startswith(b"heads_per_chunk")
+
+
+def _host_msg(lib):
+    return lib.sparse_attn_last_error()

@@ -172,6 +172,15 @@ def kept_flops(cnt, idx, N, d, bq, bk):
     return flops, tiles
 
 
+def sparsity_by_group(cnt, cfg, n_k) -> dict:
+    """Achieved block sparsity per head group of the workload (sink, near-uniform, field)."""
+    per_head = 1.0 - cnt.double().sum(dim=(0, 2)) / float(cnt.shape[0] * cnt.shape[2] * n_k)
+    groups = {"sink": list(cfg.sink_heads), "uniform": list(cfg.uniform_heads)}
+    rest = [h for h in range(cnt.shape[1]) if h not in cfg.sink_heads and h not in cfg.uniform_heads]
+    groups["field"] = rest
+    return {g: float(per_head[hs].mean().item()) for g, hs in groups.items() if hs}
+
+
 def aggregate_over_ranks(ms_step: float, flops: float, world: int, device):
     """Whole-job figures of a weak-scaled run: the slowest rank's step time and
     the kept-tile FLOPs summed over ranks (every rank takes the same two
@@ -422,6 +431,9 @@ def run_ours(args):
         check_device_error(dev)
         peaks = measured_peaks()
         fwd_tflops = fl / (fwd_ms * 1e-3) / 1e12
+        def full_tile_flops(n_tiles):
+            return 4.0 * bq * bk * d * n_tiles
+
         mask_bytes = 2.0 * B * H * N * d * 2 + 4.0 * (tiles + B * H * n_q)
         mask_gbs = mask_bytes / (mask_ms * 1e-3) / 1e9
         tr = profiled_traffic("fwd", FWD_SOURCES)
@@ -430,7 +442,12 @@ def run_ours(args):
                             "dense_fwd": dense_ms},
             "block_sparsity": sparsity,
             "kept_tiles": tiles,
-            "kept_tile_tflops": {"fwd": fwd_tflops, "step": fl / (ms_step * 1e-3) / 1e12},
+            "kept_tile_tflops": {"fwd": fwd_tflops, "step": fl / (ms_step * 1e-3) / 1e12,
+                                 "fwd_full_tiles": full_tile_flops(tiles) / (fwd_ms * 1e-3) / 1e12,
+                                 "counting": "fwd and step count valid query rows x valid keys of "
+                                             "every kept block; fwd_full_tiles counts every kept "
+                                             "block as a full bq x bk tile"},
+            "block_sparsity_by_head_group": sparsity_by_group(out["cnt"], cfg, n_k),
             "speedup_vs_own_dense": None if dense_ms is None else {
                 "fwd_only": dense_ms / fwd_ms, "mask_plus_fwd": dense_ms / (mask_ms + fwd_ms),
                 "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - sparsity)},

@@ -241,6 +241,13 @@ __device__ __forceinline__ int list_entry(const Params& prm, int r, int cnt, int
     return prm.dense ? e : __ldg(prm.idx + (size_t)r * prm.n_k + e);
 }
 
+// Index-list entry e of row r without the count check (-1 past n_k): loaded a
+// row ahead, before the row's count is known, and masked with it at use.
+__device__ __forceinline__ int raw_entry(const Params& prm, int r, int e) {
+    if (r >= prm.rows || e >= prm.n_k) return -1;
+    return prm.dense ? e : __ldg(prm.idx + (size_t)r * prm.n_k + e);
+}
+
 // Ticket lock that hands the tensor pipe to one issuer's batch at a time.
 __device__ __forceinline__ bool issue_acquire(Ctrl& C, int& ticket, volatile int* abort_flag, uint64_t lim) {
     if (!ISSUE_LOCK) return true;
@@ -327,8 +334,18 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         int k = 0, kq = 0;
         bool ok = true;
-        for (int r = blockIdx.x * NSLOT + s; ok && r < prm.rows; r += P) {
-            const int cnt = row_count(prm, r);
+        // The next row's count and first 64 index entries are loaded a row ahead.
+        const int r_first = blockIdx.x * NSLOT + s;
+        int cnt_next = r_first < prm.rows ? row_count(prm, r_first) : 0;
+        int raw0_next = raw_entry(prm, r_first, lane), raw1_next = raw_entry(prm, r_first, 32 + lane);
+        for (int r = r_first; ok && r < prm.rows; r += P) {
+            const int cnt = cnt_next;
+            const int raw0 = raw0_next, raw1 = raw1_next;
+            if (r + P < prm.rows) {
+                cnt_next = row_count(prm, r + P);
+                raw0_next = raw_entry(prm, r + P, lane);
+                raw1_next = raw_entry(prm, r + P, 32 + lane);
+            }
             const int nt = (cnt + 1) / 2;
             if (nt == 0) continue;
             const int bh = r / prm.n_q, qb = r % prm.n_q;
@@ -346,8 +363,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         tma_prefetch_l2_3d(&tmQ, sl * 64, (rn % prm.n_q) * BQ, rn / prm.n_q);
             }
             ++kq;
-            int window = list_entry(prm, r, cnt, lane);          // entries [0, 32)
-            int window_next = list_entry(prm, r, cnt, 32 + lane);  // entries [32, 64)
+            int window = lane < cnt ? raw0 : -1;                 // entries [0, 32)
+            int window_next = 32 + lane < cnt ? raw1 : -1;       // entries [32, 64)
             for (int t = 0; t < nt; ++t) {
                 const int e0 = 2 * t;
                 if (e0 > 0 && (e0 & 31) == 0) {
@@ -433,8 +450,11 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             };
             int k = 0, g = 0, kq = 0, ticket = 0;
             bool ok = true;
-            for (int r = blockIdx.x * NSLOT + s; ok && r < prm.rows; r += P) {
-                const int nt = (row_count(prm, r) + 1) / 2;
+            const int r_first = blockIdx.x * NSLOT + s;
+            int cnt_next = r_first < prm.rows ? row_count(prm, r_first) : 0;   // a row ahead
+            for (int r = r_first; ok && r < prm.rows; r += P) {
+                const int nt = (cnt_next + 1) / 2;
+                if (r + P < prm.rows) cnt_next = row_count(prm, r + P);
                 if (nt == 0) continue;
                 if (!mbar_wait_bounded(&B.q_full, kq & 1, abort_flag, W_Q, lim) || !wait_chunk(k)) {
                     ok = false;
@@ -506,8 +526,18 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         auto checked = [&](int j) -> int { return (j >= 0 && j < n_k) ? j : -1; };
         int g = 0, rowc = 0;
         bool ok = true;
-        for (int r = blockIdx.x * NSLOT + s; ok && r < prm.rows; r += P) {
-            const int cnt = row_count(prm, r);
+        // The next row's count and first 64 index entries are loaded a row ahead.
+        const int r_first = blockIdx.x * NSLOT + s;
+        int cnt_next = r_first < prm.rows ? row_count(prm, r_first) : 0;
+        int raw0_next = raw_entry(prm, r_first, lane), raw1_next = raw_entry(prm, r_first, 32 + lane);
+        for (int r = r_first; ok && r < prm.rows; r += P) {
+            const int cnt = cnt_next;
+            const int raw0 = raw0_next, raw1 = raw1_next;
+            if (r + P < prm.rows) {
+                cnt_next = row_count(prm, r + P);
+                raw0_next = raw_entry(prm, r + P, lane);
+                raw1_next = raw_entry(prm, r + P, 32 + lane);
+            }
             const int nt = (cnt + 1) / 2;
             const int bh = r / prm.n_q, qb = r % prm.n_q;
             const int q_tok = qb * BQ + row;
@@ -517,8 +547,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             float l_run = 0.f;        // sum of the bf16-rounded weights: normalises O
             float l_exact = 0.f;      // sum of the unrounded weights: the log-sum-exp
             // Index-list entries, 32 at a time (one per lane), one window ahead.
-            int window = nt > 0 ? list_entry(prm, r, cnt, lane) : -1;
-            int window_next = nt > 16 ? list_entry(prm, r, cnt, 32 + lane) : -1;
+            int window = lane < cnt ? raw0 : -1;
+            int window_next = 32 + lane < cnt ? raw1 : -1;
             for (int t = 0; t < nt; ++t) {
                 const int e0 = 2 * t;
                 if (e0 > 0 && (e0 & 31) == 0) {

@@ -129,7 +129,8 @@ EncodeTiledFn encode_fn() {
 }
 
 // [BH, N, d] bf16 viewed as a 3-D tensor (d, N, BH); box = 64 channels x
-// `rows` tokens x 1 head, 128-byte swizzle; out-of-range rows read as zero.
+// `rows` tokens x 1 head, 128-byte swizzle; out-of-range rows read as zero
+// (and are not written by a store).
 sa_status make_map(CUtensorMap* map, const void* base, const Dims& g, int rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -201,11 +202,15 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
                         const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
                         cudaStream_t st) {
     using L = sa::attn::Layout<D>;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     sa_status s;
     if ((s = make_map(&mq, Q, g, sa::attn::MROWS)) != SA_OK) return s;
     if ((s = make_map(&mk, K, g, sa::attn::BK)) != SA_OK) return s;
     if ((s = make_map(&mv, V, g, sa::attn::BK)) != SA_OK) return s;
+    // bf16 O is written by tile stores of 64 channels x one query block; the
+    // fp32 output is written directly (the map is then unused).
+    if (out_f32) mo = mq;
+    else if ((s = make_map(&mo, O, g, BQ)) != SA_OK) return s;
     auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ>;
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
                         "sparse_attn_fwd_kernel shared-memory attribute")) != SA_OK)
@@ -233,7 +238,7 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
     // Persistent: one CTA per multiprocessor (fewer when there are fewer row pairs).
     const int pairs = (prm.rows + sa::attn::NSLOT - 1) / sa::attn::NSLOT;
     const int grid = pairs < sm_count() ? pairs : sm_count();
-    kern<<<grid, sa::attn::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, prm);
+    kern<<<grid, sa::attn::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, mo, prm);
     return cuda_check(cudaGetLastError(), "sparse_attn_fwd_kernel launch");
 }
 

@@ -131,7 +131,7 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, watts = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in self.rows:
             try:
@@ -141,6 +141,7 @@ class ClockSampler:
             mx = mclk
             if pw > 300.0:  # under load
                 sm.append(clk)
+                watts.append(pw)
                 for n, v in zip(names, r[5:9]):
                     if v.lower().startswith("active"):
                         reasons.add(n)
@@ -151,7 +152,8 @@ class ClockSampler:
                 except ValueError:
                     pass
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(self.rows)}
+                "reasons": sorted(reasons), "samples": len(self.rows),
+                "power_w": statistics.median(watts) if watts else None}
 
 
 # ------------------------------------------------------------- workload
@@ -430,6 +432,13 @@ def run_ours(args):
         e2e_ms = a.elapsed_time(b) / e2e_reps
         check_device_error(dev)
         peaks = measured_peaks()
+        # The attention kernel is timed in loops of back-to-back launches that
+        # run at the board's power cap (sw_power_cap in the clock record), so
+        # its denominator is the sustained GEMM figure, measured the same way;
+        # the fraction of the burst figure is reported beside it.
+        peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+        peak_src = peaks["source"] + (" (sustained: back-to-back loop at the power cap)"
+                                      if peaks.get("bf16_tflops_sustained") else " (burst)")
         fwd_tflops = fl / (fwd_ms * 1e-3) / 1e12
         def full_tile_flops(n_tiles):
             return 4.0 * bq * bk * d * n_tiles
@@ -456,16 +465,16 @@ def run_ours(args):
                 "k": k, "p": 0.0, "block_sparsity": s95, "kept_tiles": tiles95,
                 "ms_per_call": {"mask": mask95_ms, "fwd": fwd95_ms},
                 "kept_tile_tflops_fwd": fl95 / (fwd95_ms * 1e-3) / 1e12,
-                "frac_of_bf16_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / measured_peaks()["bf16_tflops"],
+                "frac_of_bf16_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / peak_tf,
+                "frac_of_bf16_burst_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                 "speedup_vs_own_dense": None if dense_ms is None else {
                     "fwd_only": dense_ms / fwd95_ms, "mask_plus_fwd": dense_ms / (mask95_ms + fwd95_ms),
                     "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - s95)}},
-            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": fwd_tflops / peaks["bf16_tflops"],
+            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": fwd_tflops / peak_tf,
                          "traffic": None if tr is None else tr["bytes_per_launch"],
-                         "kernel": "sparse_attn_fwd_kernel", "peak_source": peaks["source"] + " (burst)",
-                         "frac_of_sustained": None if not peaks.get("bf16_tflops_sustained") else
-                         fwd_tflops / peaks["bf16_tflops_sustained"]},
+                         "kernel": "sparse_attn_fwd_kernel", "peak_source": peak_src,
+                         "frac_of_burst": fwd_tflops / peaks["bf16_tflops"]},
             "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": peaks["hbm_gbs"],
                               "unit": "GB/s", "frac": mask_gbs / peaks["hbm_gbs"],
                               "algorithmic_bytes": mask_bytes,

@@ -119,6 +119,55 @@ def test_fwd_arbitrary_lists_empty_rows_and_odd_counts(N, d, bq):
     assert np.all(O_gpu.float().cpu().numpy()[empty] == 0)
 
 
+def _aligned_qkv(alphas, N=1024, d=128, seed=11):
+    """Q rows near one direction u; the K rows of key blocks 5, 9 and 12 are
+    alpha_h * u (head h), the others random: scores against those blocks sit
+    about alpha_h * d * log2(e) / sqrt(d) above the rest (in log2 units)."""
+    g = torch.Generator().manual_seed(seed)
+    H = len(alphas)
+    u = torch.randn(d, generator=g)
+    Q = u + 0.1 * torch.randn(1, H, N, d, generator=g)
+    K = torch.randn(1, H, N, d, generator=g)
+    for h, a in enumerate(alphas):
+        for j in (5, 9, 12):
+            K[0, h, j * 64:(j + 1) * 64] = a * u + 0.1 * torch.randn(64, d, generator=g)
+    V = torch.randn(1, H, N, d, generator=g)
+    return [x.to(torch.bfloat16) for x in (Q, K, V)]
+
+
+@pytest.mark.parametrize("bq", [128, 64])
+def test_fwd_running_max_jumps(bq):
+    """Rows whose scores jump far above the running max after the first tile
+    (in log2 units): by ~50 (the weights stay against the old max, up to
+    2^53), by ~120 and ~415 (past 2^64: the tile's max is taken, O rescaled and
+    the tile recomputed), and rows whose first tile holds the largest scores."""
+    alphas = [2.5, 6.0, 20.0]
+    Qh, Kh, Vh = _aligned_qkv(alphas)
+    B, H, N, d = Qh.shape
+    n_q, n_k = -(-N // bq), -(-N // 64)
+    lists = [[0, 1, 5, 9, 12, 14], [0, 1, 2, 3, 9], [5, 0, 1, 2, 3], [2, 3, 4, 6, 7, 8, 10, 11, 12]]
+    cnt = np.zeros((B, H, n_q), dtype=np.int32)
+    idx = np.full((B, H, n_q, n_k), -1, dtype=np.int32)
+    for h in range(H):
+        for i in range(n_q):
+            li = lists[(h + i) % len(lists)]
+            cnt[0, h, i] = len(li)
+            idx[0, h, i, :len(li)] = li
+    Q, K, V = (x.cuda() for x in (Qh, Kh, Vh))
+    O_gpu, lse = sparse_attn_fwd(Q, K, V, torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(),
+                                 bq, 64, want_lse=True, out_dtype=torch.float32)
+    O_bf16 = sparse_attn_fwd(Q, K, V, torch.from_numpy(cnt).cuda(), torch.from_numpy(idx).cuda(), bq, 64)
+    check_device_error()
+    assert torch.equal(O_bf16, O_gpu.to(torch.bfloat16))
+    rows = all_rows(B, H, n_q)
+    O_ref, L_ref = O.block_sparse_attention(Qh, Kh, Vh, cnt, idx, bq, 64, rows=rows)
+    mx, mean = compare_outputs(O_gpu, O_ref, rows, bq, N)
+    lerr = float(np.max(np.abs(lse.cpu().numpy() - L_ref)))
+    print(f"\n[running-max jumps bq={bq}] max_abs={mx:.3e} mean_abs={mean:.3e} lse_max_abs={lerr:.3e}")
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, (mx, mean)
+    assert lerr < 1e-3
+
+
 def test_fwd_bad_index_is_reported_and_skipped():
     B, H, N, d, bq = 1, 2, 640, 128, 128
     Q, K, V, Qh, Kh, Vh = _custom_case(B, H, N, d, bq, seed=3)

@@ -131,9 +131,16 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=5)
+        return self.summarize(self.rows)
+
+    @staticmethod
+    def summarize(rows) -> dict:
+        """Median SM clock and board power under load (samples above 300 W, or
+        every sample if none is), the maximum SM clock, and every throttle
+        reason seen active. `rows`: the split CSV fields of FIELDS."""
         sm, mx, reasons, watts = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in self.rows:
+        for r in rows:
             try:
                 clk, mclk, pw = float(r[1]), float(r[2]), float(r[3])
             except ValueError:
@@ -146,13 +153,13 @@ class ClockSampler:
                     if v.lower().startswith("active"):
                         reasons.add(n)
         if not sm:  # short runs: fall back to every sample
-            for r in self.rows:
+            for r in rows:
                 try:
                     sm.append(float(r[1]))
                 except ValueError:
                     pass
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(self.rows),
+                "reasons": sorted(reasons), "samples": len(rows),
                 "power_w": statistics.median(watts) if watts else None}
 
 

@@ -13,7 +13,9 @@ Sources (gist.science summaries; cited by page title and section):
   Masking and Distillation Fine-Tuning" (Hindi and Arabic summaries):
   §1 Problem Statement (the Top-k and Top-p rules and their failure modes),
   §2A Hybrid Top-k + Top-p Masking (per-row union), §2C Efficient Kernel
-  Implementation (block-level mask over tiles, masked tiles skipped).
+  Implementation (block-level mask over tiles, masked tiles skipped), and
+  §2B Velocity Distillation Fine-Tuning (the sparse attention is trained
+  through, hence its backward pass in ``sparse_attn_backward``).
 * "SLA2: Sparse-Linear Attention with Learnable Routing and QAT": §1 Problem
   Statement and §2B Learnable Router (a compressed score computed from pooled
   queries and keys).
@@ -22,9 +24,10 @@ Sources (gist.science summaries; cited by page title and section):
   blocks) and §2B Centroid-Based Top-p Selection (sort by score, take items
   until the cumulative score reaches p).
 
-Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
-(closed forms, hand rows under ``tests/golden/``, invariants, library special
-cases, brute force on tiny inputs). The absolute values of the score matrix
+Parity pins: every forward function here is pinned by
+``tests/test_oracle_pins.py`` (closed forms, hand rows under ``tests/golden/``,
+invariants, library special cases, brute force on tiny inputs), the backward
+pass by ``tests/test_oracle_backward.py``. The absolute values of the score matrix
 and of the output on the synthetic workloads have no printed counterpart on
 the pages; beyond those pins they are fixed only by the definitions.
 """
@@ -41,9 +44,11 @@ from .sparse_attn_oracle import (
     block_sparse_attention,
     row_sample,
 )
+from .sparse_attn_backward import attend_row_backward, block_sparse_attention_backward
 
 __all__ = [
     "to_f64", "pool_blocks", "block_scores", "topk_count", "topp_threshold",
     "select_row", "hybrid_select", "hybrid_mask", "attend_row",
-    "block_sparse_attention", "row_sample",
+    "block_sparse_attention", "row_sample", "attend_row_backward",
+    "block_sparse_attention_backward",
 ]

@@ -229,32 +229,47 @@ def time_events(fn, reps: int, stream) -> list:
 
 
 # ----------------------------------------------------------- cpu oracle
-def oracle_sample(cfg, Qh, Kh, Vh, k, p, heads, q_stride, budget_s=None):
-    """Run the CPU oracle on a bounded sample; returns (seconds, kept FLOPs, description)."""
+def oracle_head_sample(cfg, Qh, Kh, Vh, k, p, h, rows_per_head=16):
+    """The CPU oracle on one head of the workload: the block mask of the whole
+    head, then the attention of `rows_per_head` query blocks spread evenly over
+    it. Returns (seconds, kept-tile FLOPs of the attended rows, description).
+    The same sample serves the cpu_baseline leg and the reference arm."""
     import numpy as np
     import oracle as O
     t0 = time.perf_counter()
+    q_stride = max(1, cfg.n_q // rows_per_head)
     flops = 0.0
     rows_done = 0
-    for h in heads:
-        q = O.to_f64(Qh[0, h])
-        kk = O.to_f64(Kh[0, h])
-        v = O.to_f64(Vh[0, h])
-        P = O.block_scores(O.pool_blocks(q, cfg.bq), O.pool_blocks(kk, cfg.bk), cfg.d)
-        cnt, idx, _ = O.hybrid_select(P.astype(np.float32), k, p)
-        for i in range(0, cfg.n_q, q_stride):
-            lo, hi = i * cfg.bq, min(cfg.N, (i + 1) * cfg.bq)
-            kept = idx[i, :cnt[i]]
-            O.attend_row(q[lo:hi], kk, v, kept, cfg.bk)
-            nkeys = sum(min(cfg.bk, cfg.N - j * cfg.bk) for j in kept)
-            flops += 4.0 * cfg.d * (hi - lo) * nkeys
-            rows_done += 1
-            if budget_s is not None and time.perf_counter() - t0 > budget_s:
-                break
+    q = O.to_f64(Qh[0, h])
+    kk = O.to_f64(Kh[0, h])
+    v = O.to_f64(Vh[0, h])
+    P = O.block_scores(O.pool_blocks(q, cfg.bq), O.pool_blocks(kk, cfg.bk), cfg.d)
+    cnt, idx, _ = O.hybrid_select(P.astype(np.float32), k, p)
+    for i in range(0, cfg.n_q, q_stride):
+        lo, hi = i * cfg.bq, min(cfg.N, (i + 1) * cfg.bq)
+        kept = idx[i, :cnt[i]]
+        O.attend_row(q[lo:hi], kk, v, kept, cfg.bk)
+        nkeys = sum(min(cfg.bk, cfg.N - j * cfg.bk) for j in kept)
+        flops += 4.0 * cfg.d * (hi - lo) * nkeys
+        rows_done += 1
     dt = time.perf_counter() - t0
-    desc = (f"{cfg.name}: heads {list(heads)} (mask of the whole head, then attention for every "
-            f"{q_stride}th query block: {rows_done} rows), fp64 numpy")
+    desc = (f"{cfg.name}, one head per sample: the mask of the whole head, then the attention of every "
+            f"{q_stride}th query block ({rows_done} rows); fp64 numpy")
     return dt, flops, desc
+
+
+def oracle_baseline(cfg, Qh, Kh, Vh, k, p, budget_s: float):
+    """cpu_baseline: oracle_head_sample on heads 0, 1, 2, ... until `budget_s`
+    seconds of CPU work have run (whole heads only)."""
+    total_t, total_f, heads, desc = 0.0, 0.0, [], ""
+    for h in range(cfg.H):
+        dt, fl, desc = oracle_head_sample(cfg, Qh, Kh, Vh, k, p, h)
+        total_t += dt
+        total_f += fl
+        heads.append(h)
+        if total_t > budget_s:
+            break
+    return total_t, total_f, f"heads {heads}; " + desc
 
 
 def cpu_threads() -> int:
@@ -289,14 +304,11 @@ def run_reference(args):
     Q, K, V = make_qkv(cfg, device=dev)
     Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
     del Q, K, V
-    heads_all = list(range(cfg.H))
-    q_stride = max(1, cfg.n_q // 4)
     times, flops = [], []
     desc = ""
-    for s in range(args.warmup + args.steps):
-        h = heads_all[s % cfg.H]
-        dt, fl, desc = oracle_sample(cfg, Qh, Kh, Vh, k, p, [h], q_stride)
-        if s >= args.warmup:
+    for st in range(args.warmup + args.steps):
+        dt, fl, desc = oracle_head_sample(cfg, Qh, Kh, Vh, k, p, st % cfg.H)
+        if st >= args.warmup:
             times.append(dt)
             flops.append(fl)
     value = sum(flops) / sum(times) / 1e12
@@ -308,7 +320,7 @@ def run_reference(args):
             "config": {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "N": cfg.N, "d": cfg.d,
                        "bq": cfg.bq, "bk": cfg.bk, "k": k, "p": p},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                             "sample": "per step one head (cycling): " + desc},
+                             "sample": "per step one head (heads cycling from 0): " + desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -371,25 +383,36 @@ def run_ours(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    # The timed region: K steps back to back. Events between the launches of
+    # every step time the mask and the forward inside the same loop, so the
+    # per-kernel figures and the step time come from one regime and the
+    # forward's time cannot exceed the step's.
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        do_mask()
+        ev[i][1].record(stream)
+        do_fwd()
+        ev[i][2].record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms_step = e0.elapsed_time(e1) / max(args.steps, 1)
+    mask_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev) if ev else float("nan")
+    fwd_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev) if ev else float("nan")
     ms_step, total_flops = aggregate_over_ranks(ms_step, fl, world, dev)
     value = total_flops / (ms_step * 1e-3) / 1e12
 
     extra = {}
     if not args.only_step:
-        reps = 10
-        mask_ms = statistics.median(time_events(do_mask, reps, stream))
-        fwd_ms = statistics.median(time_events(do_fwd, reps, stream))
+        peaks = measured_peaks()
+        burst = peaks["bf16_tflops"]
+        sustained = peaks.get("bf16_tflops_sustained")
         dense_ms = None
         if not args.no_dense:
             def do_dense():
@@ -397,7 +420,9 @@ def run_ours(args):
             dense_ms = statistics.median(time_events(do_dense, 3, stream))
         check_device_error(dev)
         # The ~95%-sparsity operating point: Top-k alone at the same k (p = 0)
-        # on the same inputs, where the attention does 1/20 of the dense work.
+        # on the same inputs, where the attention does 1/20 of the dense work,
+        # timed the same way (its own loop of back-to-back steps, events
+        # between the launches).
         out95 = {"cnt": torch.empty_like(out["cnt"]), "idx": torch.empty_like(out["idx"])}
         O95 = torch.empty_like(O)
 
@@ -407,10 +432,22 @@ def run_ours(args):
         def do_fwd95():
             sparse_attn_fwd(Q, K, V, out95["cnt"], out95["idx"], bq, bk, out=O95)
 
-        do_mask95()
+        for _ in range(3):
+            do_mask95()
+            do_fwd95()
+        torch.cuda.synchronize()
         fl95, tiles95 = kept_flops(out95["cnt"], out95["idx"], N, d, bq, bk)
-        mask95_ms = statistics.median(time_events(do_mask95, reps, stream))
-        fwd95_ms = statistics.median(time_events(do_fwd95, reps, stream))
+        steps95 = max(args.steps, 20)
+        ev95 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps95)]
+        for i in range(steps95):
+            ev95[i][0].record(stream)
+            do_mask95()
+            ev95[i][1].record(stream)
+            do_fwd95()
+            ev95[i][2].record(stream)
+        torch.cuda.synchronize()
+        mask95_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev95)
+        fwd95_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev95)
         check_device_error(dev)
         s95 = 1.0 - tiles95 / float(B * H * n_q * n_k)
         # End to end through the public host-buffer entry point (pinned host
@@ -438,15 +475,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_ms = a.elapsed_time(b) / e2e_reps
         check_device_error(dev)
-        peaks = measured_peaks()
-        # The attention kernel is timed in loops of back-to-back launches that
-        # run at the board's power cap (sw_power_cap in the clock record), so
-        # its denominator is the sustained GEMM figure, measured the same way;
-        # the fraction of the burst figure is reported beside it.
-        peak_tf = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
-        peak_src = peaks["source"] + (" (sustained: back-to-back loop at the power cap)"
-                                      if peaks.get("bf16_tflops_sustained") else " (burst)")
         fwd_tflops = fl / (fwd_ms * 1e-3) / 1e12
+        fwd95_tflops = fl95 / (fwd95_ms * 1e-3) / 1e12
+
         def full_tile_flops(n_tiles):
             return 4.0 * bq * bk * d * n_tiles
 
@@ -455,7 +486,9 @@ def run_ours(args):
         tr = profiled_traffic("fwd", FWD_SOURCES)
         extra = {
             "ms_per_call": {"mask": mask_ms, "fwd": fwd_ms, "mask_plus_fwd": mask_ms + fwd_ms,
-                            "dense_fwd": dense_ms},
+                            "dense_fwd": dense_ms,
+                            "timing": "mask and fwd: mean over the timed steps of the events recorded "
+                                      "between their launches; dense: median of 3 separate launches"},
             "block_sparsity": sparsity,
             "kept_tiles": tiles,
             "kept_tile_tflops": {"fwd": fwd_tflops, "step": fl / (ms_step * 1e-3) / 1e12,
@@ -469,19 +502,20 @@ def run_ours(args):
                 "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - sparsity)},
             "dense_tflops": None if dense_ms is None else dense_flops(B, H, N, d) / (dense_ms * 1e-3) / 1e12,
             "sparsity_95_point": {
-                "k": k, "p": 0.0, "block_sparsity": s95, "kept_tiles": tiles95,
+                "k": k, "p": 0.0, "block_sparsity": s95, "kept_tiles": tiles95, "steps": steps95,
                 "ms_per_call": {"mask": mask95_ms, "fwd": fwd95_ms},
-                "kept_tile_tflops_fwd": fl95 / (fwd95_ms * 1e-3) / 1e12,
-                "frac_of_bf16_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / peak_tf,
-                "frac_of_bf16_burst_peak": fl95 / (fwd95_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "kept_tile_tflops_fwd": fwd95_tflops,
+                "frac_of_bf16_burst_peak": fwd95_tflops / burst,
+                "frac_of_bf16_sustained_peak": None if not sustained else fwd95_tflops / sustained,
                 "speedup_vs_own_dense": None if dense_ms is None else {
                     "fwd_only": dense_ms / fwd95_ms, "mask_plus_fwd": dense_ms / (mask95_ms + fwd95_ms),
                     "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - s95)}},
-            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak_tf,
-                         "unit": "TFLOP/s", "frac": fwd_tflops / peak_tf,
+            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": burst,
+                         "unit": "TFLOP/s", "frac": fwd_tflops / burst,
                          "traffic": None if tr is None else tr["bytes_per_launch"],
-                         "kernel": "sparse_attn_fwd_kernel", "peak_source": peak_src,
-                         "frac_of_burst": fwd_tflops / peaks["bf16_tflops"]},
+                         "kernel": "sparse_attn_fwd_kernel",
+                         "peak_source": peaks["source"] + " bf16 dense GEMM, burst",
+                         "frac_of_sustained": None if not sustained else fwd_tflops / sustained},
             "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": peaks["hbm_gbs"],
                               "unit": "GB/s", "frac": mask_gbs / peaks["hbm_gbs"],
                               "algorithmic_bytes": mask_bytes,
@@ -493,8 +527,7 @@ def run_ours(args):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.only_step:
         Qh, Kh, Vh = Q.cpu(), K.cpu(), V.cpu()
-        heads = sorted({min(H - 1, h) for h in (0, 5, 10, 15, 25, 35)})
-        dt, cfl, desc = oracle_sample(cfg, Qh, Kh, Vh, k, p, heads, max(1, n_q // 64), budget_s=30.0)
+        dt, cfl, desc = oracle_baseline(cfg, Qh, Kh, Vh, k, p, budget_s=15.0)
         extra["cpu_baseline"] = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": cpu_threads(),
                                  "kind": "oracle", "sample": desc, "seconds": dt}
 

@@ -6,9 +6,9 @@ package is its Python binding. Build the library with ``build.build()``.
 from .capi import (EXPORTED, SparseAttnError, check_device_error, host_workspace_bytes,
                    load_library, mask_workspace_bytes, num_blocks, sparse_attn, sparse_attn_fwd,
                    sparse_attn_fwd_dense, sparse_attn_host, sparse_attn_mask, sparse_attn_select,
-                   topk_count, version)
+                   version)
 
 __all__ = ["EXPORTED", "SparseAttnError", "check_device_error", "host_workspace_bytes",
            "load_library", "mask_workspace_bytes", "num_blocks", "sparse_attn", "sparse_attn_fwd",
            "sparse_attn_fwd_dense", "sparse_attn_host", "sparse_attn_mask", "sparse_attn_select",
-           "topk_count", "version"]
+           "version"]

@@ -8,7 +8,6 @@ be present, otherwise these functions raise.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 import threading
 from typing import Optional
@@ -28,7 +27,7 @@ EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn
             "sparse_attn_select",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
             "sparse_attn_host", "sparse_attn_check_device_error",
-            "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_exp2_poly")
+            "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_fwd_withheld_copy")
 
 
 class SaShape(ctypes.Structure):
@@ -82,8 +81,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_check_device_error.restype = ctypes.c_int
         lib.sparse_attn_last_error.argtypes = []
         lib.sparse_attn_last_error.restype = ctypes.c_char_p
-        lib.sparse_attn_test_exp2_poly.argtypes = [vp, vp, ctypes.c_int64, vp]
-        lib.sparse_attn_test_exp2_poly.restype = ctypes.c_int
+        lib.sparse_attn_test_fwd_withheld_copy.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, ctypes.c_int,
+                                                           ctypes.c_uint64, vp]
+        lib.sparse_attn_test_fwd_withheld_copy.restype = ctypes.c_int
         lib.sparse_attn_version.argtypes = []
         lib.sparse_attn_version.restype = ctypes.c_char_p
         _lib = lib
@@ -129,6 +129,24 @@ def mask_workspace_bytes(B, H, N, d, bq, bk) -> int:
     return int(load_library().sparse_attn_mask_workspace_bytes(ctypes.byref(shape)))
 
 
+def _check_out(out: dict, name: str, shape, dtype: torch.dtype, device: torch.device) -> None:
+    t = out.get(name)
+    if t is None:
+        return
+    if (not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != tuple(shape)
+            or t.device != device or not t.is_contiguous()):
+        raise ValueError(f"out['{name}'] must be a contiguous {dtype} tensor of shape "
+                         f"{tuple(shape)} on {device}")
+
+
+def _check_mask_outputs(out: dict, B: int, H: int, n_q: int, n_k: int, device: torch.device) -> None:
+    """Caller-provided outputs of the mask: the kernels write them without bounds checks."""
+    _check_out(out, "cnt", (B, H, n_q), torch.int32, device)
+    _check_out(out, "idx", (B, H, n_q, n_k), torch.int32, device)
+    _check_out(out, "mask", (B, H, n_q, n_k), torch.uint8, device)
+    _check_out(out, "P", (B, H, n_q, n_k), torch.float32, device)
+
+
 def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: float, p: float, *,
                      want_mask: bool = False, want_P: bool = False, out: Optional[dict] = None,
                      workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
@@ -145,6 +163,7 @@ def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: floa
     dev = Q.device
     shape = make_shape(B, H, N, d, bq, bk)
     res = dict(out) if out is not None else {}
+    _check_mask_outputs(res, B, H, n_q, n_k, dev)
     if "cnt" not in res:
         res["cnt"] = torch.empty((B, H, n_q), dtype=torch.int32, device=dev)
     if "idx" not in res:
@@ -153,9 +172,12 @@ def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: floa
         res["mask"] = torch.empty((B, H, n_q, n_k), dtype=torch.uint8, device=dev)
     if want_P and "P" not in res:
         res["P"] = torch.empty((B, H, n_q, n_k), dtype=torch.float32, device=dev)
+    nbytes = int(lib.sparse_attn_mask_workspace_bytes(ctypes.byref(shape)))
     if workspace is None:
-        nbytes = int(lib.sparse_attn_mask_workspace_bytes(ctypes.byref(shape)))
         workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    elif (workspace.device != dev or not workspace.is_contiguous()
+          or workspace.numel() * workspace.element_size() < nbytes):
+        raise ValueError(f"workspace must be a contiguous tensor of at least {nbytes} bytes on {dev}")
     st = lib.sparse_attn_mask(ctypes.byref(shape), _ptr(Q), _ptr(K), float(k), float(p),
                               _ptr(res["cnt"]), _ptr(res["idx"]), _ptr(res.get("mask")),
                               _ptr(res.get("P")), _ptr(workspace), _stream(dev, stream))
@@ -163,7 +185,24 @@ def sparse_attn_mask(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: floa
     return res
 
 
-NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+def _header_constant(name: str) -> int:
+    """An integer macro of include/sparse_attn.h, read from the header itself."""
+    import re
+    path = os.path.join(os.path.dirname(PKG_DIR), "include", "sparse_attn.h")
+    with open(path) as f:
+        m = re.search(r"#define\s+" + name + r"\s+\(([^)]*)\)", f.read())
+    if m is None:
+        raise RuntimeError(f"{name} is not defined in {path}")
+    expr = m.group(1).replace("u", "")
+    if not re.fullmatch(r"[0-9 *]+", expr):
+        raise RuntimeError(f"{name}: unexpected definition {m.group(1)!r}")
+    value = 1
+    for factor in expr.split("*"):
+        value *= int(factor)
+    return value
+
+
+NOALLOC_SCRATCH_BYTES = _header_constant("SPARSE_ATTN_NOALLOC_SCRATCH_BYTES")
 
 
 def sparse_attn_mask_noalloc(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, k: float,
@@ -179,6 +218,10 @@ def sparse_attn_mask_noalloc(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int,
     _check_qkv(Q, K)
     lib = load_library()
     B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    if "cnt" not in out or "idx" not in out:
+        raise ValueError("out must hold 'cnt' and 'idx' (this entry point allocates nothing)")
+    _check_mask_outputs(out, B, H, n_q, n_k, Q.device)
     shape = make_shape(B, H, N, d, bq, bk)
     st = lib.sparse_attn_mask_noalloc(ctypes.byref(shape), _ptr(Q), _ptr(K), float(k), float(p),
                                       _ptr(out["cnt"]), _ptr(out["idx"]), _ptr(out.get("mask")),
@@ -328,23 +371,6 @@ def check_device_error(device=None, stream=None) -> None:
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     st = load_library().sparse_attn_check_device_error(_stream(dev, stream))
     _check("sparse_attn_check_device_error", st)
-
-
-def topk_count(k: float, n_k: int) -> int:
-    """Host copy of the library's Top-k count rule, for reporting only."""
-    if k >= 1.0:
-        return n_k
-    return min(n_k, max(0, math.ceil(k * n_k - 1e-9)))
-
-
-def exp2_poly_probe(x: torch.Tensor, stream=None) -> torch.Tensor:
-    """The attention kernel's software 2^x, evaluated on a CUDA fp32 tensor (test hook)."""
-    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
-        raise ValueError("x must be a contiguous fp32 CUDA tensor")
-    y = torch.empty_like(x)
-    st = load_library().sparse_attn_test_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x.device, stream))
-    _check("sparse_attn_test_exp2_poly", st)
-    return y
 
 
 def version() -> str:

@@ -127,6 +127,10 @@ struct Params {
     int out_f32;         // 1: O is fp32, 0: bf16 (round to nearest even)
     float scale_log2;    // log2(e) / sqrt(d)
     unsigned long long wait_limit_ns;
+    // Failure-detection test only: 1 makes the producer of slot 0 of CTA 0
+    // skip the copy of its first K tile (nothing is armed or issued for it),
+    // so that the waits depending on it run out. 0 in every normal launch.
+    int withhold_first_k;
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
@@ -134,23 +138,6 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
 }
 __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t addr, uint32_t slab_bytes) {
     return make_sdesc_sw128(addr, slab_bytes, 1024u);
-}
-
-// 2^x on the FMA pipe for x <= 8 (Cody-Waite range reduction x = n + f with
-// n = round(x), f in [-1/2, 1/2], and a degree-3 Remez polynomial for 2^f of
-// relative error 7.5e-5; coefficients from csrc/gen_exp2_poly.py). Inputs
-// below -125 are clamped (their weight is far below bf16 resolution); -inf
-// gives exactly 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-    const float xc = fmaxf(x, -125.0f);
-    const float t = xc + 12582912.0f;            // 1.5 * 2^23: round to an integer
-    const float f = xc - (t - 12582912.0f);      // f in [-1/2, 1/2]
-    float pf = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
-    pf = fmaf(pf, f, 6.932609677e-01f);
-    pf = fmaf(pf, f, 9.999280572e-01f);
-    // bits(t) << 23 equals round(x) << 23: the low 9 bits of bits(1.5*2^23) are zero.
-    const float r = __uint_as_float(__float_as_uint(pf) + (__float_as_uint(t) << 23));
-    return (x == -INFINITY) ? 0.f : r;
 }
 
 // Shared-memory descriptors as (low, high) word pairs: moving the start
@@ -407,7 +394,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                                          W_CH_EMPTY, lim);
                         if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }
                     }
-                    if (lane == 0) {
+                    const bool withheld = prm.withhold_first_k && k == 0 && s == 0 && blockIdx.x == 0;
+                    if (lane == 0 && !withheld) {
                         const CUtensorMap* map = kv ? &tmV : &tmK;
                         uint8_t* dst = sCH + c * L::CH_BYTES;
                         mbar_arrive_expect_tx(&B.ch_full[c], L::CH_BYTES);

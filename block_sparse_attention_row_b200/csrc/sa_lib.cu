@@ -197,10 +197,16 @@ int sm_count() {
     return cached[dev];
 }
 
+// Knobs of the failure-detection test hook; normal launches use the defaults.
+struct AttnTestKnobs {
+    unsigned long long wait_limit_ns = WAIT_LIMIT_NS;
+    int withhold_first_k = 0;
+};
+
 template <int D, int BQ>
 sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                         const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
-                        cudaStream_t st) {
+                        cudaStream_t st, const AttnTestKnobs& knobs) {
     using L = sa::attn::Layout<D>;
     CUtensorMap mq, mk, mv, mo;
     sa_status s;
@@ -234,7 +240,8 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
     prm.dense = dense ? 1 : 0;
     prm.out_f32 = out_f32 ? 1 : 0;
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    prm.wait_limit_ns = knobs.wait_limit_ns;
+    prm.withhold_first_k = knobs.withhold_first_k;
     // Persistent: one CTA per multiprocessor (fewer when there are fewer row pairs).
     const int pairs = (prm.rows + sa::attn::NSLOT - 1) / sa::attn::NSLOT;
     const int grid = pairs < sm_count() ? pairs : sm_count();
@@ -244,14 +251,14 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
 
 sa_status launch_fwd(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                      const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
-                     cudaStream_t st) {
+                     cudaStream_t st, const AttnTestKnobs& knobs = AttnTestKnobs()) {
     if (g.d == 128 && g.bq == 128)
-        return launch_attn_t<128, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<128, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st, knobs);
     if (g.d == 128 && g.bq == 64)
-        return launch_attn_t<128, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<128, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st, knobs);
     if (g.d == 64 && g.bq == 128)
-        return launch_attn_t<64, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
-    return launch_attn_t<64, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st);
+        return launch_attn_t<64, 128>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st, knobs);
+    return launch_attn_t<64, 64>(g, Q, K, V, cnt, idx, O, out_f32, lse, dense, st, knobs);
 }
 
 sa_status check_out_dtype(int o_dtype) {
@@ -260,24 +267,23 @@ sa_status check_out_dtype(int o_dtype) {
     return SA_OK;
 }
 
-__global__ void exp2_poly_probe_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) y[i] = sa::attn::exp2_poly(x[i]);
+sa_status check_fwd_args(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                         const int32_t* cnt, const int32_t* idx, void* O, int o_dtype,
+                         const float* lse_or_null, Dims& g) {
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if ((s = check_out_dtype(o_dtype)) != SA_OK) return s;
+    if (!Q || !K || !V || !cnt || !idx || !O)
+        return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, cnt, idx, O");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(cnt) || !aligned16(idx) ||
+        !aligned16(O) || (lse_or_null && !aligned16(lse_or_null)))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
+    return SA_OK;
 }
 
 }  // namespace
 
 extern "C" {
-
-sa_status sparse_attn_test_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-    if (!x || !y || n < 0) return fail(SA_ERR_INVALID_ARG, "exp2 probe: bad arguments");
-    if (n == 0) return ok();
-    const int64_t blocks = (n + 255) / 256;
-    if (blocks > 0x7FFFFFFF) return fail(SA_ERR_INVALID_ARG, "exp2 probe: n too large");
-    exp2_poly_probe_kernel<<<(unsigned)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
-    sa_status s = cuda_check(cudaGetLastError(), "exp2 probe launch");
-    return s != SA_OK ? s : ok();
-}
 
 size_t sparse_attn_mask_workspace_bytes(const sa_shape* shape) {
     Dims g;
@@ -386,15 +392,28 @@ sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, c
                           float* lse_or_null, void* stream) {
     Dims g;
     sa_status s;
-    if ((s = check_shape(shape, g)) != SA_OK) return s;
-    if ((s = check_out_dtype(o_dtype)) != SA_OK) return s;
-    if (!Q || !K || !V || !cnt || !idx || !O)
-        return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, cnt, idx, O");
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(cnt) || !aligned16(idx) ||
-        !aligned16(O) || (lse_or_null && !aligned16(lse_or_null)))
-        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
+    if ((s = check_fwd_args(shape, Q, K, V, cnt, idx, O, o_dtype, lse_or_null, g)) != SA_OK) return s;
     s = launch_fwd(g, Q, K, V, cnt, idx, O, o_dtype == SA_F32, lse_or_null, false,
                    reinterpret_cast<cudaStream_t>(stream));
+    if (s != SA_OK) return s;
+    return ok();
+}
+
+sa_status sparse_attn_test_fwd_withheld_copy(const sa_shape* shape, const void* Q, const void* K,
+                                             const void* V, const int32_t* cnt, const int32_t* idx,
+                                             void* O, int o_dtype, uint64_t wait_limit_ns,
+                                             void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_fwd_args(shape, Q, K, V, cnt, idx, O, o_dtype, nullptr, g)) != SA_OK) return s;
+    if (wait_limit_ns < 1000000ull || wait_limit_ns > WAIT_LIMIT_NS)
+        return fail(SA_ERR_INVALID_ARG, "wait_limit_ns=%llu outside [1e6, 4e9]",
+                    (unsigned long long)wait_limit_ns);
+    AttnTestKnobs knobs;
+    knobs.wait_limit_ns = wait_limit_ns;
+    knobs.withhold_first_k = 1;
+    s = launch_fwd(g, Q, K, V, cnt, idx, O, o_dtype == SA_F32, nullptr, false,
+                   reinterpret_cast<cudaStream_t>(stream), knobs);
     if (s != SA_OK) return s;
     return ok();
 }

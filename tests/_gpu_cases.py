@@ -62,10 +62,11 @@ def flip_report(P_gpu: np.ndarray, P_ref: np.ndarray, k: float, p: float) -> dic
 
     A differing row is a near tie if two scores straddling either row's
     selection boundary lie within 1e-6 of each other, or if the cumulative
-    mass at the boundary lies within 1e-6 of the target. It is "explained by
-    score rounding" if the same holds with 1e-6 replaced by the row's largest
-    |P_gpu - P_ref| times the row length (the most that rounding of the scores
-    can move either quantity).
+    mass at the boundary lies within 1e-6 of the target (SpargeAttention2 §2A:
+    the Top-p prefix is decided by where the cumulative mass reaches p). Every
+    other differing row is listed in "not_near_tie" and fails the parity gate;
+    "rounding_sized" counts those of them whose gap is below the row's largest
+    |P_gpu - P_ref| times the row length, for diagnosis only.
     """
     n_k = P_gpu.shape[-1]
     Pg = P_gpu.reshape(-1, n_k).astype(np.float32)
@@ -73,10 +74,9 @@ def flip_report(P_gpu: np.ndarray, P_ref: np.ndarray, k: float, p: float) -> dic
     cg, ig, mg = O.hybrid_select(Pg, k, p)
     cr, ir, mr = O.hybrid_select(Pr, k, p)
     rows = np.nonzero(np.any(mg != mr, axis=1))[0]
-    near, explained, unexplained = 0, 0, []
+    near, rounding_sized, not_near = 0, 0, []
     for r in rows:
         eps_row = float(np.max(np.abs(Pg[r].astype(np.float64) - Pr[r].astype(np.float64))))
-        tol_explain = max(NEAR_TIE, 2.0 * eps_row * n_k)
         order = np.lexsort((np.arange(n_k), -Pg[r].view(np.uint32).astype(np.int64)))
         vals = Pg[r][order].astype(np.float64)
         L = int(cg[r])
@@ -92,12 +92,12 @@ def flip_report(P_gpu: np.ndarray, P_ref: np.ndarray, k: float, p: float) -> dic
         cum_gap = min(abs(cum[m] - Tm) for m in range(max(lo - 1, 0), min(hi + 1, n_k))) / 2.0 ** 31
         if min_gap < NEAR_TIE or cum_gap < NEAR_TIE:
             near += 1
-        elif min_gap < tol_explain or cum_gap < tol_explain:
-            explained += 1
         else:
-            unexplained.append(int(r))
+            not_near.append(int(r))
+            if min(min_gap, cum_gap) < 2.0 * eps_row * n_k:
+                rounding_sized += 1
     return {"rows": int(Pg.shape[0]), "differing": int(rows.size), "near_tie": near,
-            "explained_by_score_rounding": explained, "unexplained": unexplained,
+            "not_near_tie": not_near, "rounding_sized": rounding_sized,
             "max_abs_dP": float(np.max(np.abs(Pg.astype(np.float64) - Pr.astype(np.float64))))}
 
 

@@ -100,32 +100,6 @@ def test_binding_refuses_cpu_tensors():
         sparse_attn_mask(q, q, 64, 64, 0.1, 0.9)
 
 
-def test_topk_count_matches_oracle_rule():
-    import oracle
-    from block_sparse_attention_row_b200 import topk_count
-    for k in (0.0, 0.03, 0.05, 0.07, 0.1, 0.125, 0.25, 0.5, 0.999, 1.0):
-        for n in (1, 7, 64, 100, 256, 275, 512, 1182):
-            assert topk_count(k, n) == oracle.topk_count(k, n)
-
-
-def test_exp2_poly_constants_come_from_the_remez_script():
-    """The kernel's polynomial constants are the ones the derivation script prints."""
-    import importlib.util
-    spec = importlib.util.spec_from_file_location(
-        "gen_exp2_poly", os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "gen_exp2_poly.py"))
-    gen = importlib.util.module_from_spec(spec)
-    spec.loader.exec_module(gen)
-    coef, err = gen.remez_relative()
-    assert err < 1e-4
-    src = open(os.path.join(ROOT, "block_sparse_attention_row_b200", "csrc", "sa_attn_kernel.cuh")).read()
-    body = src[src.index("float exp2_poly("):src.index("return (x == -INFINITY)")]
-    lits = [float(v) for v in re.findall(r"([0-9]\.[0-9]+e[-+][0-9]+)f", body)]
-    assert len(lits) == 4
-    c3, c2, c1, c0 = lits
-    import numpy as np
-    assert np.allclose([c0, c1, c2, c3], np.float32(coef), rtol=0, atol=2e-9)
-
-
 def test_host_pipeline_workspace_and_validation(lib):
     """sparse_attn_host: chunk planning and host-side argument checks (nothing enqueued)."""
     from block_sparse_attention_row_b200.capi import host_workspace_bytes, make_shape
@@ -158,3 +132,30 @@ def test_host_pipeline_workspace_and_validation(lib):
 
 def _host_msg(lib):
     return lib.sparse_attn_last_error()
+
+
+def test_mask_output_validation_rejects_wrong_tensors():
+    """The caller-provided outputs of the mask are checked before any launch
+    (the kernels write them without bounds checks)."""
+    import torch
+    from block_sparse_attention_row_b200 import capi
+    dev = torch.device("cpu")
+    good = {"cnt": torch.empty(1, 2, 8, dtype=torch.int32), "idx": torch.empty(1, 2, 8, 16, dtype=torch.int32),
+            "mask": torch.empty(1, 2, 8, 16, dtype=torch.uint8), "P": torch.empty(1, 2, 8, 16)}
+    capi._check_mask_outputs(good, 1, 2, 8, 16, dev)
+    bad = [("cnt", torch.empty(1, 2, 9, dtype=torch.int32)),            # wrong shape
+           ("idx", torch.empty(1, 2, 8, 16, dtype=torch.int64)),        # wrong dtype
+           ("mask", torch.empty(1, 2, 16, 8, dtype=torch.uint8).transpose(-1, -2)),  # not contiguous
+           ("P", torch.empty(1, 2, 8, 15))]
+    for name, t in bad:
+        with pytest.raises(ValueError, match=name):
+            capi._check_mask_outputs({**good, name: t}, 1, 2, 8, 16, dev)
+    with pytest.raises(ValueError, match="on cuda"):
+        capi._check_mask_outputs(good, 1, 2, 8, 16, torch.device("cuda", 0))
+
+
+def test_noalloc_scratch_size_is_read_from_the_header():
+    from block_sparse_attention_row_b200 import capi
+    src = open(HEADERS[0]).read()
+    assert "#define SPARSE_ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)" in src
+    assert capi.NOALLOC_SCRATCH_BYTES == 32 * 1024 * 1024

@@ -54,7 +54,7 @@ def test_fwd_matches_oracle(name, stride):
     assert lerr < 1e-4
 
 
-@pytest.mark.parametrize("k,p", [(0.03, 0.80), (0.05, 0.90), (0.10, 0.95)])
+@pytest.mark.parametrize("k,p", CONFIGS["sweep"].kp)
 def test_fwd_matches_oracle_sweep(k, p):
     mx, mean, _ = _run("sweep", k, p, 8)
     assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL
@@ -217,17 +217,3 @@ def test_fwd_is_deterministic():
     b = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], cfg.bq, cfg.bk)
     check_device_error()
     assert torch.equal(a, b)
-
-
-def test_software_exp2_within_its_bound():
-    """The FMA-pipe 2^x used for a quarter of the softmax: relative error < 1e-4
-    over the arguments the kernel produces (x <= 8), exact 0 at -inf."""
-    from block_sparse_attention_row_b200.capi import exp2_poly_probe
-    x = torch.cat([torch.linspace(-124.0, 8.0, 2_000_001, dtype=torch.float64),
-                   torch.tensor([0.0, -0.5, 0.5, -1e-30, 8.0, -20.25])]).float().cuda()
-    y = exp2_poly_probe(x).double()
-    ref = torch.exp2(x.double())
-    rel = ((y - ref).abs() / ref).max().item()
-    assert rel < 1e-4, rel
-    z = exp2_poly_probe(torch.tensor([-float("inf")], device="cuda"))
-    assert z.item() == 0.0

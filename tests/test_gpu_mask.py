@@ -3,7 +3,12 @@
 Bit-exact: the oracle's selection applied to the GPU-written fp32 scores must
 equal the GPU's cnt / idx / mask on every row of every workload. Near ties
 between the GPU scores and the oracle's own fp64 scores are counted and
-reported; a differing row that no rounding of the scores explains fails.
+reported; a differing row that is not a near tie (two straddling scores, or the
+boundary mass, within 1e-6) fails.
+
+Score accuracy: the GPU's fp32 softmax of the block logits is within 2e-6 of
+the oracle's fp64 scores elementwise (measured: at most 4.8e-7 on the five
+workloads), and each row sums to 1 within 2e-6 (fp64 sum).
 """
 import json
 
@@ -37,7 +42,8 @@ def test_mask_bit_exact_on_gpu_scores(name, k, p, record_property):
     assert_same_selection(m["cnt"].cpu().numpy(), m["idx"].cpu().numpy(), m["mask"].cpu().numpy(),
                           cnt_o, idx_o, mask_o)
     # Rows of P are probability distributions.
-    assert np.all(P_gpu >= 0) and np.allclose(P_gpu.sum(-1), 1.0, atol=1e-4)
+    assert np.all(P_gpu >= 0)
+    assert np.max(np.abs(P_gpu.sum(-1, dtype=np.float64) - 1.0)) < 2e-6
     # Near-tie accounting against the oracle's own scores.
     P_ref = reference_scores(Qh, Kh, cfg.bq, cfg.bk)
     rep = flip_report(P_gpu, P_ref, k, p)
@@ -45,8 +51,8 @@ def test_mask_bit_exact_on_gpu_scores(name, k, p, record_property):
     rep["block_sparsity"] = sparsity
     record_property("near_tie_report", json.dumps(rep))
     print(f"\n[{name} k={k} p={p}] {json.dumps(rep)}")
-    assert rep["unexplained"] == [], rep
-    assert rep["max_abs_dP"] < 1e-4
+    assert rep["not_near_tie"] == [], rep
+    assert rep["max_abs_dP"] < 2e-6, rep
 
 
 @pytest.mark.parametrize("N,d,bq", [(300, 64, 64), (300, 128, 128), (1000, 128, 128), (4097, 64, 128),

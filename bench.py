@@ -450,6 +450,56 @@ def run_ours(args):
         fwd95_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev95)
         check_device_error(dev)
         s95 = 1.0 - tiles95 / float(B * H * n_q * n_k)
+        # Backward pass and the FP8 forward, each timed in its own loop of
+        # back-to-back launches with events between them (as above), at the
+        # workload's (k, p) and at the 95% point.
+        from block_sparse_attention_row_b200 import (bwd_workspace_bytes, sparse_attn_bwd, sparse_attn_fwd_fp8,
+                                                     sparse_attn_quantize_fp8)
+        from synth import make_grad_out
+        dO = make_grad_out(B, H, N, d, seed=cfg.seed + 7, device=dev)
+        bws = torch.empty(bwd_workspace_bytes(B, H, N, d, bq, bk), dtype=torch.uint8, device=dev)
+        grads = {n: torch.empty(Q.shape, dtype=torch.bfloat16, device=dev) for n in ("dQ", "dK", "dV")}
+        lse_buf = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        q8 = sparse_attn_quantize_fp8(Q, K, bq, bk) if d == 128 else None
+        O8 = torch.empty_like(O)
+
+        def loop_time(fns, reps):
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(fns) + 1)] for _ in range(reps)]
+            for i in range(reps):
+                for j, fn in enumerate(fns):
+                    evs[i][j].record(stream)
+                    fn()
+                evs[i][-1].record(stream)
+            torch.cuda.synchronize()
+            return [statistics.fmean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(len(fns))]
+
+        extra_paths = {}
+        for tag, mo in (("config", out), ("sparsity_95_point", out95)):
+            fl_t, tiles_t = kept_flops(mo["cnt"], mo["idx"], N, d, bq, bk)
+            sparse_attn_fwd(Q, K, V, mo["cnt"], mo["idx"], bq, bk, out=O, lse=lse_buf, want_lse=True)
+
+            def do_bwd():
+                sparse_attn_bwd(Q, K, V, O, dO, lse_buf, mo["cnt"], mo["idx"], bq, bk, out_dtype=torch.bfloat16,
+                                out=grads, workspace=bws)
+            for _ in range(2):
+                do_bwd()
+            bwd_ms, = loop_time([do_bwd], max(5, min(args.steps, 10)))
+            entry = {"bwd_ms": bwd_ms, "bwd_kept_tile_tflops": 2.5 * fl_t / (bwd_ms * 1e-3) / 1e12,
+                     "bwd_frac_of_bf16_burst_peak": 2.5 * fl_t / (bwd_ms * 1e-3) / 1e12 / burst}
+            if q8 is not None:
+                def do_q8():
+                    sparse_attn_quantize_fp8(Q, K, bq, bk, out=q8)
+
+                def do_f8():
+                    sparse_attn_fwd_fp8(q8, V, mo["cnt"], mo["idx"], bq, bk, out=O8)
+                for _ in range(2):
+                    do_q8()
+                    do_f8()
+                qms, f8ms = loop_time([do_q8, do_f8], max(10, min(args.steps, 20)))
+                entry.update({"fp8_quantize_ms": qms, "fp8_fwd_ms": f8ms,
+                              "fp8_fwd_kept_tile_tflops": fl_t / (f8ms * 1e-3) / 1e12})
+            extra_paths[tag] = entry
+        check_device_error(dev)
         # End to end through the public host-buffer entry point (pinned host
         # Q, K, V in; O back in host memory): the library pipelines the copies
         # with the mask and attention by chunks of heads.
@@ -520,6 +570,10 @@ def run_ours(args):
                               "unit": "GB/s", "frac": mask_gbs / peaks["hbm_gbs"],
                               "algorithmic_bytes": mask_bytes,
                               "kernels": "pool_kernel + score_kernel + select_kernel"},
+            "backward_and_fp8": dict(extra_paths, counting=(
+                "bwd: 2.5 x the kept-tile FLOPs of the forward (the five products dV, dP, S, dQ, dK per "
+                "kept pair against the forward's two; the kernels compute S and dP twice, which is not "
+                "counted); bf16 gradients; fp8: per-block e4m3 Q and K, bf16 P V")),
             "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         }

@@ -3,12 +3,14 @@
 The compute lives in libsparse_attn.so (C ABI: include/sparse_attn.h); this
 package is its Python binding. Build the library with ``build.build()``.
 """
-from .capi import (EXPORTED, SparseAttnError, check_device_error, host_workspace_bytes,
+from .capi import (EXPORTED, SparseAttnError, bwd_workspace_bytes, check_device_error, host_workspace_bytes,
                    load_library, mask_workspace_bytes, num_blocks, sparse_attn, sparse_attn_fwd,
-                   sparse_attn_fwd_dense, sparse_attn_host, sparse_attn_mask, sparse_attn_select,
+                   sparse_attn_bwd, sparse_attn_fwd_dense, sparse_attn_host, sparse_attn_mask,
+                   sparse_attn_select, sparse_attn_quantize_fp8, sparse_attn_fwd_fp8,
                    version)
 
-__all__ = ["EXPORTED", "SparseAttnError", "check_device_error", "host_workspace_bytes",
+__all__ = ["EXPORTED", "SparseAttnError", "bwd_workspace_bytes", "check_device_error", "sparse_attn_bwd", "host_workspace_bytes",
            "load_library", "mask_workspace_bytes", "num_blocks", "sparse_attn", "sparse_attn_fwd",
            "sparse_attn_fwd_dense", "sparse_attn_host", "sparse_attn_mask", "sparse_attn_select",
+           "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8",
            "version"]

@@ -13,7 +13,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libsparse_attn.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["sa_lib.cu"]
-DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_attn_kernel.cuh",
+DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_attn_kernel.cuh", "sa_bwd_kernels.cuh", "sa_fp8_kernels.cuh",
         "sa_status_codes.h"]
 
 
@@ -35,7 +35,8 @@ def is_stale() -> bool:
     if not os.path.exists(LIB_PATH):
         return True
     t = os.path.getmtime(LIB_PATH)
-    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(INCLUDE, "sparse_attn.h")]
+    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(INCLUDE, h) for h in
+                                                    ("sparse_attn.h", "sparse_attn_testing.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 

@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 
 # Every entry point declared in include/sparse_attn.h and include/sparse_attn_testing.h.
 EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_mask_noalloc",
-            "sparse_attn_select",
+            "sparse_attn_select", "sparse_attn_bwd_workspace_bytes", "sparse_attn_bwd",
+            "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
             "sparse_attn_host", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_fwd_withheld_copy")
@@ -72,6 +73,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_fwd.restype = ctypes.c_int
         lib.sparse_attn_fwd_dense.argtypes = [sp, vp, vp, vp, vp, ctypes.c_int, f32p, vp]
         lib.sparse_attn_fwd_dense.restype = ctypes.c_int
+        lib.sparse_attn_bwd_workspace_bytes.argtypes = [sp]
+        lib.sparse_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_bwd.argtypes = [sp, vp, vp, vp, vp, vp, f32p, i32p, i32p, vp, vp, vp, ctypes.c_int, vp, vp]
+        lib.sparse_attn_bwd.restype = ctypes.c_int
+        lib.sparse_attn_quantize_fp8.argtypes = [sp, vp, vp, vp, vp, f32p, f32p, vp]
+        lib.sparse_attn_quantize_fp8.restype = ctypes.c_int
+        lib.sparse_attn_fwd_fp8.argtypes = [sp, vp, vp, f32p, f32p, vp, i32p, i32p, vp, ctypes.c_int, f32p, vp]
+        lib.sparse_attn_fwd_fp8.restype = ctypes.c_int
         lib.sparse_attn_host_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
         lib.sparse_attn_host_workspace_bytes.restype = ctypes.c_size_t
         lib.sparse_attn_host.argtypes = [sp, vp, vp, vp, ctypes.c_double, ctypes.c_double, vp, ctypes.c_int,
@@ -304,6 +313,102 @@ def sparse_attn_fwd_dense(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bq:
                                    _stream(Q.device, stream))
     _check("sparse_attn_fwd_dense", st)
     return (O, lse) if want_lse else O
+
+
+def sparse_attn_quantize_fp8(Q: torch.Tensor, K: torch.Tensor, bq: int, bk: int, *, out: Optional[dict] = None,
+                             stream=None) -> dict:
+    """Per-block e4m3 codes of Q and K: {'Q8', 'K8' (uint8 [B,H,N,d]), 'q_scale'
+    fp32 [B,H,n_q], 'k_scale' fp32 [B,H,n_k]}; x is approximately code * scale."""
+    _check_qkv(Q, K)
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = Q.device
+    res = dict(out) if out is not None else {}
+    for name, shp, dt in (("Q8", Q.shape, torch.uint8), ("K8", Q.shape, torch.uint8),
+                          ("q_scale", (B, H, n_q), torch.float32), ("k_scale", (B, H, n_k), torch.float32)):
+        if name in res:
+            _check_out(res, name, shp, dt, dev)
+        else:
+            res[name] = torch.empty(shp, dtype=dt, device=dev)
+    shape = make_shape(B, H, N, d, bq, bk)
+    st = load_library().sparse_attn_quantize_fp8(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(res["Q8"]),
+                                                 _ptr(res["K8"]), _ptr(res["q_scale"]), _ptr(res["k_scale"]),
+                                                 _stream(dev, stream))
+    _check("sparse_attn_quantize_fp8", st)
+    return res
+
+
+def sparse_attn_fwd_fp8(q8: dict, V: torch.Tensor, cnt: torch.Tensor, idx: torch.Tensor, bq: int, bk: int, *,
+                        want_lse: bool = False, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16, stream=None):
+    """Block-sparse attention with the score product in FP8: q8 is the dict of
+    sparse_attn_quantize_fp8; V bf16. Returns O (, lse)."""
+    _check_qkv(V)
+    B, H, N, d = V.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = V.device
+    for name, shp, dt in (("Q8", V.shape, torch.uint8), ("K8", V.shape, torch.uint8),
+                          ("q_scale", (B, H, n_q), torch.float32), ("k_scale", (B, H, n_k), torch.float32)):
+        if name not in q8:
+            raise ValueError(f"q8 must hold '{name}'")
+        _check_out(q8, name, shp, dt, dev)
+    for t, shp in ((cnt, (B, H, n_q)), (idx, (B, H, n_q, n_k))):
+        if t.dtype != torch.int32 or not t.is_contiguous() or tuple(t.shape) != shp or t.device != dev:
+            raise ValueError(f"index tensor must be contiguous int32 {shp} on {dev}")
+    O = _out_tensor(V, out, out_dtype)
+    if want_lse and lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    shape = make_shape(B, H, N, d, bq, bk)
+    st = load_library().sparse_attn_fwd_fp8(ctypes.byref(shape), _ptr(q8["Q8"]), _ptr(q8["K8"]),
+                                            _ptr(q8["q_scale"]), _ptr(q8["k_scale"]), _ptr(V), _ptr(cnt),
+                                            _ptr(idx), _ptr(O), SA_F32 if O.dtype == torch.float32 else SA_BF16,
+                                            _ptr(lse), _stream(dev, stream))
+    _check("sparse_attn_fwd_fp8", st)
+    return (O, lse) if want_lse else O
+
+
+def bwd_workspace_bytes(B, H, N, d, bq, bk) -> int:
+    shape = make_shape(B, H, N, d, bq, bk)
+    return int(load_library().sparse_attn_bwd_workspace_bytes(ctypes.byref(shape)))
+
+
+def sparse_attn_bwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, O: torch.Tensor, dO: torch.Tensor,
+                    lse: torch.Tensor, cnt: torch.Tensor, idx: torch.Tensor, bq: int, bk: int, *,
+                    out_dtype: torch.dtype = torch.float32, out: Optional[dict] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dQ, dK, dV) of sparse_attn_fwd for the upstream gradient dO,
+    with the kept-block lists held fixed. O and lse are the forward's bf16
+    output and log-sum-exp. Outputs are fp32 (default) or bf16."""
+    _check_qkv(Q, K, V, O, dO)
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = Q.device
+    for t, shp, dt in ((cnt, (B, H, n_q), torch.int32), (idx, (B, H, n_q, n_k), torch.int32),
+                       (lse, (B, H, N), torch.float32)):
+        if t.dtype != dt or not t.is_contiguous() or tuple(t.shape) != shp or t.device != dev:
+            raise ValueError(f"cnt, idx, lse must be contiguous {dt} {shp} on {dev}")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    res = dict(out) if out is not None else {}
+    for name in ("dQ", "dK", "dV"):
+        if name in res:
+            _check_out(res, name, Q.shape, out_dtype, dev)
+        else:
+            res[name] = torch.empty(Q.shape, dtype=out_dtype, device=dev)
+    lib = load_library()
+    shape = make_shape(B, H, N, d, bq, bk)
+    nbytes = int(lib.sparse_attn_bwd_workspace_bytes(ctypes.byref(shape)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    elif (workspace.device != dev or not workspace.is_contiguous()
+          or workspace.numel() * workspace.element_size() < nbytes):
+        raise ValueError(f"workspace must be a contiguous tensor of at least {nbytes} bytes on {dev}")
+    st = lib.sparse_attn_bwd(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(lse),
+                             _ptr(cnt), _ptr(idx), _ptr(res["dQ"]), _ptr(res["dK"]), _ptr(res["dV"]),
+                             SA_F32 if out_dtype == torch.float32 else SA_BF16, _ptr(workspace),
+                             _stream(dev, stream))
+    _check("sparse_attn_bwd", st)
+    return res["dQ"], res["dK"], res["dV"]
 
 
 def sparse_attn(Q, K, V, bq: int, bk: int, k: float, p: float, *, stream=None):

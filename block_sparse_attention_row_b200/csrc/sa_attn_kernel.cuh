@@ -79,11 +79,17 @@ enum WaitSite : unsigned int {
     W_S_FULL = 0xE005, W_O_FULL = 0xE006, W_Q_EMPTY = 0xE007, W_LOCK = 0xE008, W_STG = 0xE009
 };
 
-template <int D>
+// FP8: Q and K are e4m3 codes (one byte per element, 128 channels per
+// 128-byte slab) with per-block scales; V stays bf16.
+template <int D, bool FP8 = false>
 struct Layout {
-    static constexpr int SLABS = D / 64;                 // 64-channel (128-byte) slabs
-    static constexpr int Q_BYTES = MROWS * D * 2;        // one Q tile
-    static constexpr int CH_BYTES = TILE_N * D * 2;      // one K or V tile
+    static constexpr int SLABS = D / 64;                 // 64-channel (128-byte) bf16 slabs: V, O
+    static constexpr int QK_SLABS = FP8 ? D / 128 : D / 64;   // 128-byte slabs of Q and K
+    static constexpr int QK_CH = FP8 ? 128 : 64;         // channels per Q/K slab
+    static constexpr int Q_BYTES = MROWS * D * (FP8 ? 1 : 2);   // one Q tile
+    static constexpr int K_BYTES = TILE_N * D * (FP8 ? 1 : 2);  // one K tile
+    static constexpr int CH_BYTES = TILE_N * D * 2;      // one chunk slot: a V tile or a K tile
+    static_assert(!FP8 || D == 128, "the FP8 path is built for d = 128");
     static constexpr int NCH = (D == 128) ? 2 : 4;       // chunk ring depth per slot
     static constexpr int SLOT_BYTES = Q_BYTES + NCH * CH_BYTES;
     // Per slot, the staging tile of the bf16 epilogue: 128 rows x 64 channels.
@@ -131,6 +137,9 @@ struct Params {
     // skip the copy of its first K tile (nothing is armed or issued for it),
     // so that the waits depending on it run out. 0 in every normal launch.
     int withhold_first_k;
+    // FP8 path: per-block scales of the Q and K codes (null otherwise).
+    const float* q_scale;   // [BH * n_q]
+    const float* k_scale;   // [BH * n_k]
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
@@ -190,6 +199,22 @@ __device__ __forceinline__ void umma_ss_batch<4>(uint32_t d, const uint64_t (&a)
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, p1;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, p1;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, p1;\n\t}" ::"r"(d),
+        "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+        "r"(idesc), "r"(acc0)
+        : "memory");
+}
+
+// Four SS MMAs of kind::f8f6f4 (e4m3 A and B, K = 32 each) into one accumulator.
+__device__ __forceinline__ void umma_ss_batch_f8x4(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                                   uint32_t idesc, uint32_t acc0) {
+    asm volatile(
+        "{\n\t.reg .pred p0, p1;\n\t"
+        "setp.ne.b32 p0, %10, 0;\n\t"
+        "setp.eq.b32 p1, %9, %9;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %9, p0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %9, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %9, p1;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %9, p1;\n\t}" ::"r"(d),
         "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
         "r"(idesc), "r"(acc0)
         : "memory");
@@ -273,12 +298,12 @@ __device__ __forceinline__ void issue_release(Ctrl& C, int ticket) {
     *reinterpret_cast<volatile int*>(&C.ticket_serving) = ticket + 1;
 }
 
-template <int D, int BQ>
+template <int D, int BQ, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        const Params prm) {
-    using L = Layout<D>;
+    using L = Layout<D, FP8>;
     constexpr int NCH = L::NCH;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -359,12 +384,12 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             }
             if (lane == 0) {
                 mbar_arrive_expect_tx(&B.q_full, L::Q_BYTES);
-                for (int sl = 0; sl < L::SLABS; ++sl)
-                    tma_load_3d(sQ + sl * (MROWS * 128), &tmQ, &B.q_full, sl * 64, qb * BQ, bh);
+                for (int sl = 0; sl < L::QK_SLABS; ++sl)
+                    tma_load_3d(sQ + sl * (MROWS * 128), &tmQ, &B.q_full, sl * L::QK_CH, qb * BQ, bh);
                 const int rn = r + P;   // the slot's next row: its Q tile into L2 now
                 if (rn < prm.rows)
-                    for (int sl = 0; sl < L::SLABS; ++sl)
-                        tma_prefetch_l2_3d(&tmQ, sl * 64, (rn % prm.n_q) * BQ, rn / prm.n_q);
+                    for (int sl = 0; sl < L::QK_SLABS; ++sl)
+                        tma_prefetch_l2_3d(&tmQ, sl * L::QK_CH, (rn % prm.n_q) * BQ, rn / prm.n_q);
             }
             ++kq;
             int window = lane < cnt ? raw0 : -1;                 // entries [0, 32)
@@ -398,11 +423,13 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     if (lane == 0 && !withheld) {
                         const CUtensorMap* map = kv ? &tmV : &tmK;
                         uint8_t* dst = sCH + c * L::CH_BYTES;
-                        mbar_arrive_expect_tx(&B.ch_full[c], L::CH_BYTES);
-                        for (int sl = 0; sl < L::SLABS; ++sl) {
+                        const int nsl = kv ? L::SLABS : L::QK_SLABS;
+                        const int sch = kv ? 64 : L::QK_CH;
+                        mbar_arrive_expect_tx(&B.ch_full[c], kv ? L::CH_BYTES : L::K_BYTES);
+                        for (int sl = 0; sl < nsl; ++sl) {
                             uint8_t* base = dst + sl * (TILE_N * 128);
-                            tma_load_3d(base, map, &B.ch_full[c], sl * 64, r0, bh);
-                            tma_load_3d(base + BK * 128, map, &B.ch_full[c], sl * 64, r1, bh);
+                            tma_load_3d(base, map, &B.ch_full[c], sl * sch, r0, bh);
+                            tma_load_3d(base + BK * 128, map, &B.ch_full[c], sl * sch, r1, bh);
                         }
                     }
                     ++k;
@@ -428,7 +455,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int s = warp - MMA_WARP;
         SlotBars& B = C.sb[s];
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = make_idesc_bf16(MROWS, TILE_N, false);
+            constexpr uint32_t IDESC_S = FP8 ? make_idesc_e4m3(MROWS, TILE_N) : make_idesc_bf16(MROWS, TILE_N, false);
             constexpr uint32_t IDESC_PV = make_idesc_bf16(MROWS, D, true);
             uint8_t* sQ = smem + s * L::SLOT_BYTES;
             uint8_t* sCH = sQ + L::Q_BYTES;
@@ -440,15 +467,16 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             // S_s = Q_s K^T from the K tile in chunk c.
             auto issue_s = [&](int c) {
                 const Desc kd = {k_desc.lo + ((uint32_t)(c * L::CH_BYTES) >> 4), k_desc.hi};
-                uint64_t ad[L::SLABS * 4], bd[L::SLABS * 4];
+                uint64_t ad[L::QK_SLABS * 4], bd[L::QK_SLABS * 4];
 #pragma unroll
-                for (int sl = 0; sl < L::SLABS; ++sl)
+                for (int sl = 0; sl < L::QK_SLABS; ++sl)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         ad[sl * 4 + kk] = desc_at(q_desc, (sl * (MROWS * 128) + kk * 32) >> 4);
                         bd[sl * 4 + kk] = desc_at(kd, (sl * (TILE_N * 128) + kk * 32) >> 4);
                     }
-                umma_ss_batch<L::SLABS * 4>(tS, ad, bd, IDESC_S, 0u);
+                if constexpr (FP8) umma_ss_batch_f8x4(tS, ad, bd, IDESC_S, 0u);
+                else umma_ss_batch<L::QK_SLABS * 4>(tS, ad, bd, IDESC_S, 0u);
             };
             auto wait_chunk = [&](int kk) -> bool {
                 return mbar_wait_spin(&B.ch_full[kk % NCH], (kk / NCH) & 1, abort_flag, W_CH_FULL, lim);
@@ -549,6 +577,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const int q_tok = qb * BQ + row;
             const bool row_valid = (row < BQ) && (q_tok < prm.N);
             const size_t out_off = ((size_t)bh * prm.N + q_tok) * D;
+            // FP8: scale of this query block's Q codes (the key blocks' scales are read per tile).
+            const float row_sq = FP8 ? __ldg(prm.q_scale + (size_t)bh * prm.n_q + qb) : 1.f;
             float m_run = -INFINITY;  // running max, log2 units, as used for P
             float l_run = 0.f;        // sum of the bf16-rounded weights: normalises O
             float l_exact = 0.f;      // sum of the unrounded weights: the log-sum-exp
@@ -572,6 +602,16 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 // Valid key columns: [0, v0) from block j0, [64, 64 + v1) from j1.
                 const int v0 = j0 < 0 ? 0 : min(BK, prm.N - j0 * BK);
                 const int v1 = j1 < 0 ? 0 : min(BK, prm.N - j1 * BK);
+                // Exponent scale of each half of the tile: log2(e)/sqrt(d), times
+                // the Q and K block scales on the FP8 path (kept positive so that
+                // -inf padding stays -inf; a zero scale only occurs for an
+                // all-zero block, whose codes, and scores, are 0).
+                float sc0 = sl2, sc1 = sl2;
+                if constexpr (FP8) {
+                    const float* ks = prm.k_scale + (size_t)bh * n_k;
+                    sc0 = sl2 * fmaxf(row_sq * (j0 >= 0 ? __ldg(ks + j0) : 1.f), 1e-30f);
+                    sc1 = sl2 * fmaxf(row_sq * (j1 >= 0 ? __ldg(ks + j1) : 1.f), 1e-30f);
+                }
                 // The weights of a tile are taken against the running max m_run
                 // as it stands, without the tile's own max: fp32 and bf16 hold
                 // weights up to 2^MAX_WEIGHT_LOG2 without loss of relative
@@ -593,7 +633,33 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                             if (!valid) rr[c] = 0xFF800000u;
                         }
                     }
-                    if (with_max) {
+                    if (FP8 && with_max) {
+                        // Max of each half (its own scale), 8 chains of three-input max each.
+                        float mh[2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            float mc[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) mc[q] = __uint_as_float(rr[64 * h + 2 * q]);
+#pragma unroll
+                            for (int c = 64 * h + 16; c < 64 * h + 64; c += 16) {
+#pragma unroll
+                                for (int q = 0; q < 8; ++q)
+                                    mc[q] = max3f(mc[q], __uint_as_float(rr[c + 2 * q]), __uint_as_float(rr[c + 2 * q + 1]));
+                            }
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) mc[q] = fmaxf(mc[q], __uint_as_float(rr[64 * h + 2 * q + 1]));
+                            mh[h] = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
+                                          fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
+                        }
+                        const float mx = fmaxf(mh[0] * sc0, mh[1] * sc1);
+                        if (t == 0) {
+                            m_run = mx;
+                        } else if (mx > m_run) {
+                            alpha = ex2_approx(m_run - mx);
+                            m_run = mx;
+                        }
+                    } else if (with_max) {
                         // Row max over 8 independent chains of three-input max.
                         float mc[8];
 #pragma unroll
@@ -616,7 +682,8 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                         }
                     }
                     const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                    const uint64_t scale2 = f2_pack(sl2, sl2);
+                    const uint64_t scale2 = f2_pack(sc0, sc0);
+                    const uint64_t scale2_hi = f2_pack(sc1, sc1);   // the second half (equal unless FP8)
                     const uint64_t negm2 = f2_pack(-m_use, -m_use);
                     uint64_t acc[4], acc_exact[2];
 #pragma unroll
@@ -630,7 +697,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int pc = 0; pc < TILE_N / 2; ++pc) {
                         // y = S * log2(e)/sqrt(d) - m for two columns at once.
                         const uint64_t y = f2_fma(f2_pack(__uint_as_float(rr[2 * pc]), __uint_as_float(rr[2 * pc + 1])),
-                                                  scale2, negm2);
+                                                  (FP8 && pc >= TILE_N / 4) ? scale2_hi : scale2, negm2);
                         f2_unpack(y, pe[2 * pc], pe[2 * pc + 1]);
                     }
 #pragma unroll

@@ -17,6 +17,8 @@
 #include "sa_ptx.cuh"
 #include "sa_mask_kernels.cuh"
 #include "sa_attn_kernel.cuh"
+#include "sa_bwd_kernels.cuh"
+#include "sa_fp8_kernels.cuh"
 
 namespace {
 
@@ -145,6 +147,22 @@ sa_status make_map(CUtensorMap* map, const void* base, const Dims& g, int rows) 
     return SA_OK;
 }
 
+// [BH, N, d] e4m3 codes (one byte each) viewed as (d, N, BH); box = 128
+// channels (128 bytes) x `rows` tokens x 1 head, 128-byte swizzle.
+sa_status make_map_u8(CUtensorMap* map, const void* base, const Dims& g, int rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[3] = {(cuuint64_t)g.d, (cuuint64_t)g.N, (cuuint64_t)g.BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)g.d, (cuuint64_t)g.N * g.d};
+    const cuuint32_t box[3] = {128, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (CUresult %d)", (int)r);
+    return SA_OK;
+}
+
 // ------------------------------------------------------------ launches
 template <int D>
 sa_status launch_pool_score(const Dims& g, const void* Q, const void* K, const Workspace& w,
@@ -203,21 +221,32 @@ struct AttnTestKnobs {
     int withhold_first_k = 0;
 };
 
-template <int D, int BQ>
+// The FP8 path's per-block scales (null on the bf16 path).
+struct Fp8Scales {
+    const float* q = nullptr;
+    const float* k = nullptr;
+};
+
+template <int D, int BQ, bool FP8 = false>
 sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                         const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
-                        cudaStream_t st, const AttnTestKnobs& knobs) {
-    using L = sa::attn::Layout<D>;
+                        cudaStream_t st, const AttnTestKnobs& knobs, const Fp8Scales& sc = Fp8Scales()) {
+    using L = sa::attn::Layout<D, FP8>;
     CUtensorMap mq, mk, mv, mo;
     sa_status s;
-    if ((s = make_map(&mq, Q, g, sa::attn::MROWS)) != SA_OK) return s;
-    if ((s = make_map(&mk, K, g, sa::attn::BK)) != SA_OK) return s;
+    if (FP8) {
+        if ((s = make_map_u8(&mq, Q, g, sa::attn::MROWS)) != SA_OK) return s;
+        if ((s = make_map_u8(&mk, K, g, sa::attn::BK)) != SA_OK) return s;
+    } else {
+        if ((s = make_map(&mq, Q, g, sa::attn::MROWS)) != SA_OK) return s;
+        if ((s = make_map(&mk, K, g, sa::attn::BK)) != SA_OK) return s;
+    }
     if ((s = make_map(&mv, V, g, sa::attn::BK)) != SA_OK) return s;
     // bf16 O is written by tile stores of 64 channels x one query block; the
     // fp32 output is written directly (the map is then unused).
     if (out_f32) mo = mq;
     else if ((s = make_map(&mo, O, g, BQ)) != SA_OK) return s;
-    auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ>;
+    auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ, FP8>;
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
                         "sparse_attn_fwd_kernel shared-memory attribute")) != SA_OK)
         return s;
@@ -242,6 +271,8 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     prm.wait_limit_ns = knobs.wait_limit_ns;
     prm.withhold_first_k = knobs.withhold_first_k;
+    prm.q_scale = sc.q;
+    prm.k_scale = sc.k;
     // Persistent: one CTA per multiprocessor (fewer when there are fewer row pairs).
     const int pairs = (prm.rows + sa::attn::NSLOT - 1) / sa::attn::NSLOT;
     const int grid = pairs < sm_count() ? pairs : sm_count();
@@ -281,9 +312,141 @@ sa_status check_fwd_args(const sa_shape* shape, const void* Q, const void* K, co
     return SA_OK;
 }
 
+// ------------------------------------------------------------ backward
+struct BwdWorkspace {
+    size_t lsed, bitmap, ucnt, uidx, total;
+    int nw, n_kp;
+};
+
+BwdWorkspace bwd_layout(const Dims& g) {
+    BwdWorkspace w;
+    w.nw = (g.n_k + 31) / 32;
+    w.n_kp = (g.n_k + 1) / 2;
+    w.lsed = 0;
+    w.bitmap = round256((size_t)g.BH * g.n_q * g.bq * sizeof(float2));
+    w.ucnt = w.bitmap + round256((size_t)g.BH * g.n_q * w.nw * sizeof(uint32_t));
+    w.uidx = w.ucnt + round256((size_t)g.BH * w.n_kp * sizeof(int32_t));
+    w.total = w.uidx + round256((size_t)g.BH * w.n_kp * g.n_q * sizeof(int32_t));
+    return w;
+}
+
+template <typename KernelT>
+sa_status prepare_tc_kernel(KernelT kern, int dyn_bytes, const char* name) {
+    sa_status s;
+    if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_bytes),
+                        name)) != SA_OK)
+        return s;
+    // The kernel moves registers between its warpgroups (setmaxnreg); the
+    // split adds up only for the launch register count it was written for.
+    cudaFuncAttributes fa;
+    if ((s = cuda_check(cudaFuncGetAttributes(&fa, kern), name)) != SA_OK) return s;
+    if (fa.numRegs != sa::bwd::LAUNCH_REGS)
+        return fail(SA_ERR_UNSUPPORTED, "%s was built with %d registers per thread, not %d", name, fa.numRegs,
+                    sa::bwd::LAUNCH_REGS);
+    return SA_OK;
+}
+
+template <int D, int BQ>
+sa_status launch_bwd_t(const Dims& g, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                       const float* lse, const int32_t* cnt, const int32_t* idx, void* dQ, void* dK, void* dV,
+                       bool out_f32, uint8_t* ws, cudaStream_t st) {
+    const BwdWorkspace w = bwd_layout(g);
+    float2* lsed = reinterpret_cast<float2*>(ws + w.lsed);
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws + w.bitmap);
+    int32_t* ucnt = reinterpret_cast<int32_t*>(ws + w.ucnt);
+    int32_t* uidx = reinterpret_cast<int32_t*>(ws + w.uidx);
+    sa_status s;
+    sa::bwd::bwd_rows_kernel<D><<<dim3(g.n_q, g.BH), 128, w.nw * sizeof(uint32_t), st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(O), reinterpret_cast<const __nv_bfloat16*>(dO), lse, cnt, idx, lsed,
+        bitmap, g.N, g.bq, g.n_q, g.n_k, w.nw);
+    if ((s = cuda_check(cudaGetLastError(), "bwd_rows_kernel launch")) != SA_OK) return s;
+    sa::bwd::bwd_transpose_kernel<<<dim3((w.nw + sa::bwd::TR_WARPS - 1) / sa::bwd::TR_WARPS, g.BH),
+                                    sa::bwd::TR_WARPS * 32, 0, st>>>(bitmap, ucnt, uidx, g.n_q, w.nw, w.n_kp);
+    if ((s = cuda_check(cudaGetLastError(), "bwd_transpose_kernel launch")) != SA_OK) return s;
+
+    CUtensorMap mq128, mdo128, mqb, mdob, mk, mv;
+    if ((s = make_map(&mq128, Q, g, sa::bwd::MROWS)) != SA_OK || (s = make_map(&mdo128, dO, g, sa::bwd::MROWS)) != SA_OK ||
+        (s = make_map(&mqb, Q, g, BQ)) != SA_OK || (s = make_map(&mdob, dO, g, BQ)) != SA_OK ||
+        (s = make_map(&mk, K, g, sa::bwd::BK)) != SA_OK || (s = make_map(&mv, V, g, sa::bwd::BK)) != SA_OK)
+        return s;
+    sa::bwd::Params prm;
+    prm.lsed = lsed;
+    prm.N = g.N;
+    prm.n_q = g.n_q;
+    prm.n_k = g.n_k;
+    prm.n_kp = w.n_kp;
+    prm.out_f32 = out_f32 ? 1 : 0;
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    prm.scale = (float)(1.0 / std::sqrt((double)D));
+    prm.wait_limit_ns = WAIT_LIMIT_NS;
+
+    auto kdq = sa::bwd::bwd_dq_kernel<D, BQ>;
+    constexpr int DQ_BYTES = sa::bwd::DQLayout<D, BQ>::DYN_BYTES;
+    if ((s = prepare_tc_kernel(kdq, DQ_BYTES, "bwd_dq_kernel")) != SA_OK) return s;
+    sa::bwd::Params pq = prm;
+    pq.cnt = cnt;
+    pq.idx = idx;
+    pq.out0 = dQ;
+    pq.out1 = nullptr;
+    pq.items = g.BH * g.n_q;
+    const int gq = pq.items < sm_count() ? pq.items : sm_count();
+    kdq<<<gq, sa::bwd::NUM_THREADS, DQ_BYTES, st>>>(mq128, mk, mv, mdo128, pq);
+    if ((s = cuda_check(cudaGetLastError(), "bwd_dq_kernel launch")) != SA_OK) return s;
+
+    auto kkv = sa::bwd::bwd_dkdv_kernel<D, BQ>;
+    constexpr int KV_BYTES = sa::bwd::KVLayout<D, BQ>::DYN_BYTES;
+    if ((s = prepare_tc_kernel(kkv, KV_BYTES, "bwd_dkdv_kernel")) != SA_OK) return s;
+    sa::bwd::Params pk = prm;
+    pk.cnt = ucnt;
+    pk.idx = uidx;
+    pk.out0 = dV;
+    pk.out1 = dK;
+    pk.items = g.BH * w.n_kp;
+    const int gk = pk.items < sm_count() ? pk.items : sm_count();
+    kkv<<<gk, sa::bwd::NUM_THREADS, KV_BYTES, st>>>(mqb, mk, mv, mdob, pk);
+    return cuda_check(cudaGetLastError(), "bwd_dkdv_kernel launch");
+}
+
+sa_status launch_bwd(const Dims& g, const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                     const float* lse, const int32_t* cnt, const int32_t* idx, void* dQ, void* dK, void* dV,
+                     bool out_f32, uint8_t* ws, cudaStream_t st) {
+    if (g.d == 128 && g.bq == 128)
+        return launch_bwd_t<128, 128>(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, out_f32, ws, st);
+    if (g.d == 128 && g.bq == 64)
+        return launch_bwd_t<128, 64>(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, out_f32, ws, st);
+    if (g.d == 64 && g.bq == 128)
+        return launch_bwd_t<64, 128>(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, out_f32, ws, st);
+    return launch_bwd_t<64, 64>(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, out_f32, ws, st);
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t sparse_attn_bwd_workspace_bytes(const sa_shape* shape) {
+    Dims g;
+    if (check_shape(shape, g) != SA_OK) return 0;
+    return bwd_layout(g).total;
+}
+
+sa_status sparse_attn_bwd(const sa_shape* shape, const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* lse, const int32_t* cnt, const int32_t* idx, void* dQ,
+                          void* dK, void* dV, int g_dtype, void* workspace, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if ((s = check_out_dtype(g_dtype)) != SA_OK) return s;
+    if (!Q || !K || !V || !O || !dO || !lse || !cnt || !idx || !dQ || !dK || !dV || !workspace)
+        return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, workspace");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(lse) ||
+        !aligned16(cnt) || !aligned16(idx) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required; 256 for workspace)");
+    s = launch_bwd(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, g_dtype == SA_F32,
+                   reinterpret_cast<uint8_t*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+    if (s != SA_OK) return s;
+    return ok();
+}
 
 size_t sparse_attn_mask_workspace_bytes(const sa_shape* shape) {
     Dims g;
@@ -395,6 +558,52 @@ sa_status sparse_attn_fwd(const sa_shape* shape, const void* Q, const void* K, c
     if ((s = check_fwd_args(shape, Q, K, V, cnt, idx, O, o_dtype, lse_or_null, g)) != SA_OK) return s;
     s = launch_fwd(g, Q, K, V, cnt, idx, O, o_dtype == SA_F32, lse_or_null, false,
                    reinterpret_cast<cudaStream_t>(stream));
+    if (s != SA_OK) return s;
+    return ok();
+}
+
+sa_status sparse_attn_quantize_fp8(const sa_shape* shape, const void* Q, const void* K, uint8_t* Q8, uint8_t* K8,
+                                   float* q_scale, float* k_scale, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if (!Q || !K || !Q8 || !K8 || !q_scale || !k_scale)
+        return fail(SA_ERR_INVALID_ARG, "NULL pointer among Q, K, Q8, K8, q_scale, k_scale");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(Q8) || !aligned16(K8) || !aligned16(q_scale) ||
+        !aligned16(k_scale))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    dim3 grid(g.n_q + g.n_k, g.BH);
+    auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
+    auto* k = reinterpret_cast<const __nv_bfloat16*>(K);
+    if (g.d == 128)
+        sa::fp8::quantize_kernel<128><<<grid, sa::fp8::QUANT_THREADS, 0, st>>>(q, k, Q8, K8, q_scale, k_scale, g.N,
+                                                                               g.bq, g.bk, g.n_q, g.n_k);
+    else
+        sa::fp8::quantize_kernel<64><<<grid, sa::fp8::QUANT_THREADS, 0, st>>>(q, k, Q8, K8, q_scale, k_scale, g.N,
+                                                                              g.bq, g.bk, g.n_q, g.n_k);
+    if ((s = cuda_check(cudaGetLastError(), "quantize_kernel launch")) != SA_OK) return s;
+    return ok();
+}
+
+sa_status sparse_attn_fwd_fp8(const sa_shape* shape, const uint8_t* Q8, const uint8_t* K8, const float* q_scale,
+                              const float* k_scale, const void* V, const int32_t* cnt, const int32_t* idx, void* O,
+                              int o_dtype, float* lse_or_null, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_fwd_args(shape, Q8, K8, V, cnt, idx, O, o_dtype, lse_or_null, g)) != SA_OK) return s;
+    if (g.d != 128) return fail(SA_ERR_UNSUPPORTED, "d=%d: the FP8 path supports d = 128", g.d);
+    if (!q_scale || !k_scale) return fail(SA_ERR_INVALID_ARG, "NULL q_scale or k_scale");
+    if (!aligned16(q_scale) || !aligned16(k_scale))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
+    Fp8Scales sc;
+    sc.q = q_scale;
+    sc.k = k_scale;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool f32 = o_dtype == SA_F32;
+    s = (g.bq == 128)
+            ? launch_attn_t<128, 128, true>(g, Q8, K8, V, cnt, idx, O, f32, lse_or_null, false, st, AttnTestKnobs(), sc)
+            : launch_attn_t<128, 64, true>(g, Q8, K8, V, cnt, idx, O, f32, lse_or_null, false, st, AttnTestKnobs(), sc);
     if (s != SA_OK) return s;
     return ok();
 }

@@ -155,6 +155,72 @@ sa_status sparse_attn_fwd_dense(const sa_shape* shape, const void* Q, const void
                                 const void* V, void* O, int o_dtype, float* lse_or_null,
                                 void* stream);
 
+/* Low-bit forward, step 1 of 2: per-block FP8 (e4m3) quantisation of Q and K.
+ * "SLA2: Sparse-Linear Attention with Learnable Routing and QAT" §2C runs
+ * the sparse branch in low-bit (INT8/FP8) attention; the page names neither
+ * format nor scaling. Here: one fp32 scale per query block of Q (bq tokens)
+ * and per key block of K (bk tokens), s = amax / 448 with amax the block's
+ * largest |x| (fp32); each code is e4m3(x * (448 / amax)), products and
+ * quotient in fp32 round-to-nearest, the conversion rounding to nearest even
+ * and saturating at 448. An all-zero block gets s = 0 and zero codes.
+ * Inputs:  Q, K bf16 [B,H,N,d].
+ * Outputs: Q8, K8 e4m3 codes [B,H,N,d] (one byte each); q_scale fp32
+ *          [B,H,n_q]; k_scale fp32 [B,H,n_k]. */
+sa_status sparse_attn_quantize_fp8(const sa_shape* shape, const void* Q, const void* K,
+                                   uint8_t* Q8, uint8_t* K8, float* q_scale, float* k_scale,
+                                   void* stream);
+
+/* Low-bit forward, step 2 of 2: sparse_attn_fwd with the score product in
+ * FP8. S = Q K^T runs on the tensor cores in e4m3 (tcgen05 kind::f8f6f4) and
+ * is rescaled per tile by q_scale[i] * k_scale[j]; P and V stay in the bf16
+ * path of sparse_attn_fwd (on B200 the exponentials of P already take as long
+ * per tile as the bf16 P V product, so an FP8 P V would not shorten a tile).
+ * Same kept-tile semantics, outputs and error reporting as sparse_attn_fwd.
+ * Inputs: Q8, K8, q_scale, k_scale from sparse_attn_quantize_fp8; V bf16
+ *         [B,H,N,d]; cnt, idx as for sparse_attn_fwd. d must be 128
+ *         (SA_ERR_UNSUPPORTED otherwise).
+ * Outputs: O [B,H,N,d] of type o_dtype; lse (optional) fp32 [B,H,N]. */
+sa_status sparse_attn_fwd_fp8(const sa_shape* shape, const uint8_t* Q8, const uint8_t* K8,
+                              const float* q_scale, const float* k_scale, const void* V,
+                              const int32_t* cnt, const int32_t* idx,
+                              void* O, int o_dtype, float* lse_or_null, void* stream);
+
+/* Bytes of device workspace sparse_attn_bwd needs for `shape`: the per-row
+ * log-sum-exp and D = rowsum(dO * O) (8 * B*H * n_q * bq bytes), the
+ * kept-block bitmap (4 * B*H * n_q * ceil(n_k/32)), and the transposed lists
+ * (4 * B*H * ceil(n_k/2) * (n_q + 1)), each rounded up to 256 bytes.
+ * 0 on an invalid shape. */
+size_t sparse_attn_bwd_workspace_bytes(const sa_shape* shape);
+
+/* Backward pass of step 4: the gradients of sparse_attn_fwd's output with the
+ * kept-block lists held fixed. SpargeAttention2 §2B (Velocity Distillation
+ * Fine-Tuning) fine-tunes the model through the sparse attention of §2C;
+ * the pages give no formula, so this is the plain derivative of the forward
+ * (the selection of §2A is piecewise constant in Q and K and carries none).
+ * For every query block i with kept key tokens u, c = 1/sqrt(d) and
+ * P = softmax(c Q_i K_u^T) (recomputed from lse):
+ *   dV_u += P^T dO_i;  dS = P * (dO_i V_u^T - D_i), D_i = rowsum(dO_i * O_i);
+ *   dQ_i = c dS K_u;   dK_u += c dS^T Q_i.
+ * A key token that no query block keeps gets dK = dV = 0; a query block with
+ * cnt = 0 gets dQ = 0.
+ * Inputs:  Q, K, V bf16 [B,H,N,d] (those of the forward); O bf16 [B,H,N,d]
+ *          and lse fp32 [B,H,N], the forward's bf16 output and log-sum-exp;
+ *          dO bf16 [B,H,N,d], the gradient of the loss with respect to O;
+ *          cnt, idx as given to the forward. A list must not repeat a block:
+ *          a repeated or out-of-range entry is reported as
+ *          SA_ERR_DEVICE_ASSERT and counted once (repeated) or skipped.
+ * Outputs: dQ, dK, dV [B,H,N,d] of type g_dtype (SA_BF16 or SA_F32).
+ * workspace: device buffer of sparse_attn_bwd_workspace_bytes(shape) bytes,
+ *          256-byte aligned; its contents are scratch.
+ * The sums are deterministic (no atomics): dQ is accumulated per query block
+ * in list order, dK and dV per pair of adjacent key blocks in ascending
+ * query-block order. */
+sa_status sparse_attn_bwd(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                          const void* O, const void* dO, const float* lse,
+                          const int32_t* cnt, const int32_t* idx,
+                          void* dQ, void* dK, void* dV, int g_dtype,
+                          void* workspace, void* stream);
+
 /* Bytes of device workspace sparse_attn_host needs for `shape` with chunks of
  * `heads_per_chunk` (b, h) heads (0 = the library's choice, see below): two
  * device copies of a chunk of Q, K, V and O (O in the element type o_dtype),

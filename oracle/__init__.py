@@ -45,10 +45,13 @@ from .sparse_attn_oracle import (
     row_sample,
 )
 from .sparse_attn_backward import attend_row_backward, block_sparse_attention_backward
+from .sparse_attn_fp8 import (block_sparse_attention_fp8, dequantize_blocks, e4m3_round,
+                              quantize_blocks)
 
 __all__ = [
     "to_f64", "pool_blocks", "block_scores", "topk_count", "topp_threshold",
     "select_row", "hybrid_select", "hybrid_mask", "attend_row",
     "block_sparse_attention", "row_sample", "attend_row_backward",
-    "block_sparse_attention_backward",
+    "block_sparse_attention_backward", "e4m3_round", "quantize_blocks", "dequantize_blocks",
+    "block_sparse_attention_fp8",
 ]

@@ -164,3 +164,10 @@ def make_qkv(cfg: WorkloadConfig, device="cpu"):
                            grid=cfg.grid, positional_field=cfg.positional_field,
                            sink_heads=cfg.sink_heads, uniform_heads=cfg.uniform_heads,
                            bk_sink=cfg.bk)
+
+
+def make_grad_out(B: int, H: int, N: int, d: int, *, seed: int, device="cpu") -> torch.Tensor:
+    """A seeded upstream gradient dO for the backward pass: iid N(0, 1) drawn
+    in fp32 from its own generator, rounded once to bf16, shape [B, H, N, d]."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    return torch.randn((B, H, N, d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)

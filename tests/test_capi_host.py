@@ -159,3 +159,45 @@ def test_noalloc_scratch_size_is_read_from_the_header():
     src = open(HEADERS[0]).read()
     assert "#define SPARSE_ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)" in src
     assert capi.NOALLOC_SCRATCH_BYTES == 32 * 1024 * 1024
+
+
+@pytest.mark.parametrize("B,H,N,d,bq", [(1, 2, 4096, 64, 64), (1, 40, 32760, 128, 128), (2, 24, 17550, 128, 128),
+                                        (1, 3, 777, 64, 64), (1, 1, 1, 128, 128)])
+def test_bwd_workspace_bytes(lib, B, H, N, d, bq):
+    from block_sparse_attention_row_b200.capi import make_shape
+    n_q, n_k = -(-N // bq), -(-N // 64)
+    nw, n_kp = -(-n_k // 32), -(-n_k // 2)
+    r = lambda x: (x + 255) // 256 * 256
+    want = r(B * H * n_q * bq * 8) + r(B * H * n_q * nw * 4) + r(B * H * n_kp * 4) + r(B * H * n_kp * n_q * 4)
+    assert lib.sparse_attn_bwd_workspace_bytes(ctypes.byref(make_shape(B, H, N, d, bq, 64))) == want
+    assert lib.sparse_attn_bwd_workspace_bytes(ctypes.byref(make_shape(B, H, N, 96, bq, 64))) == 0
+
+
+def test_bwd_host_validation(lib):
+    from block_sparse_attention_row_b200.capi import make_shape
+    good = ctypes.byref(make_shape(1, 2, 4096, 64, 64, 64))
+    a, z, ws = ctypes.c_void_p(16), ctypes.c_void_p(0), ctypes.c_void_p(256)
+    args = [a] * 11
+    for pos in range(11):
+        bad = list(args)
+        bad[pos] = z
+        assert lib.sparse_attn_bwd(good, *bad, 1, ws, None) == 1, pos
+    assert lib.sparse_attn_bwd(good, *args, 5, ws, None) == 1          # unknown g_dtype
+    assert lib.sparse_attn_bwd(good, *args, 1, ctypes.c_void_p(16), None) == 1   # workspace alignment
+    bad = list(args)
+    bad[3] = ctypes.c_void_p(24)
+    assert lib.sparse_attn_bwd(good, *bad, 1, ws, None) == 1
+    assert b"aligned" in lib.sparse_attn_last_error()
+
+
+def test_fp8_host_validation(lib):
+    from block_sparse_attention_row_b200.capi import make_shape
+    a, z = ctypes.c_void_p(16), ctypes.c_void_p(0)
+    d64 = ctypes.byref(make_shape(1, 2, 4096, 64, 64, 64))
+    d128 = ctypes.byref(make_shape(1, 2, 4096, 128, 128, 64))
+    assert lib.sparse_attn_fwd_fp8(d64, a, a, a, a, a, a, a, a, 0, None, None) == 2    # d = 64 unsupported
+    assert b"FP8" in lib.sparse_attn_last_error()
+    assert lib.sparse_attn_fwd_fp8(d128, a, a, z, a, a, a, a, a, 0, None, None) == 1   # no q_scale
+    assert lib.sparse_attn_fwd_fp8(d128, a, a, a, a, a, a, a, a, 3, None, None) == 1   # o_dtype
+    assert lib.sparse_attn_quantize_fp8(d128, a, a, a, z, a, a, None) == 1
+    assert lib.sparse_attn_quantize_fp8(d128, a, a, a, ctypes.c_void_p(20), a, a, None) == 1

@@ -680,6 +680,17 @@ struct HostPlan {
 
 constexpr int HOST_MIN_ROWS_PER_CHUNK = 2368;   // ~8 query-block rows per attention pipeline on 148 SMs
 
+// Heads of the next chunk when `rest` heads remain: full chunks of `hpc`
+// heads while at least two chunks' worth remain, then halving chunks. The
+// copies cross PCIe back to back while the compute of earlier chunks runs
+// under them; what the pipeline cannot hide is the compute and copy-out of
+// the last chunk, so the tail is made small.
+int chunk_heads(int rest, int hpc) {
+    if (rest >= 2 * hpc) return hpc;
+    const int c = (rest + 1) / 2;
+    return c < 1 ? 1 : (c > hpc ? hpc : c);
+}
+
 sa_status host_plan(const sa_shape* shape, int o_dtype, int heads_per_chunk, HostPlan& hp) {
     sa_status s;
     if ((s = check_shape(shape, hp.g)) != SA_OK) return s;
@@ -690,7 +701,8 @@ sa_status host_plan(const sa_shape* shape, int o_dtype, int heads_per_chunk, Hos
     if (hpc == 0) hpc = (HOST_MIN_ROWS_PER_CHUNK + g.n_q - 1) / g.n_q;
     if (hpc > g.BH) hpc = g.BH;
     hp.hpc = hpc;
-    hp.nchunk = (g.BH + hpc - 1) / hpc;
+    hp.nchunk = 0;
+    for (int bh0 = 0; bh0 < g.BH; bh0 += chunk_heads(g.BH - bh0, hpc)) ++hp.nchunk;
     hp.esize_o = (o_dtype == SA_F32) ? 4 : 2;
     const size_t tok = (size_t)hpc * g.N * g.d;
     hp.qkv_bytes = tok * 2;
@@ -794,10 +806,10 @@ sa_status sparse_attn_host(const sa_shape* shape, const void* Q, const void* K, 
         if ((s = cuda_check(cudaStreamWaitEvent(st, ev_start, 0), "order after the caller's stream")) != SA_OK)
             return s;
     const size_t tok_bytes = (size_t)g.N * g.d * 2;   // one head of Q, K or V
-    for (int c = 0; c < hp.nchunk; ++c) {
+    int bh0 = 0;
+    for (int c = 0; c < hp.nchunk; bh0 += chunk_heads(g.BH - bh0, hp.hpc), ++c) {
         const int b = c & 1;
-        const int bh0 = c * hp.hpc;
-        const int hc = (g.BH - bh0 < hp.hpc) ? g.BH - bh0 : hp.hpc;
+        const int hc = chunk_heads(g.BH - bh0, hp.hpc);
         const sa_shape sub = {1, hc, g.N, g.d, g.bq, g.bk};
         void* Qd = ws + hp.off_q[b];
         void* Kd = ws + hp.off_k[b];

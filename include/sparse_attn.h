@@ -232,13 +232,16 @@ size_t sparse_attn_host_workspace_bytes(const sa_shape* shape, int o_dtype, int 
  * buffers. It has no counterpart in the papers: it packages the same
  * computation for callers whose Q, K, V are in host memory, overlapping the
  * PCIe copies with the GPU work. The (b, h) heads are independent rows of the
- * mask and of the attention, so they are processed in chunks of
+ * mask and of the attention, so they are processed in chunks of at most
  * heads_per_chunk heads (0 = enough heads for at least 2,368 query-block rows
- * per chunk, about 8 rows per attention pipeline of a B200): while chunk c is
- * computed, chunk c+1 is copied to the device and chunk c-1's results back to
- * the host, on three streams owned by the library, with two device copies of
- * every chunk buffer (in `workspace`). The results are those of the device
- * entry points on the whole tensors, bit for bit.
+ * per chunk, about 8 rows per attention pipeline of a B200); once fewer than
+ * two full chunks remain, each chunk takes half of the remaining heads
+ * (rounded up), so that the last chunk, whose compute and copy-out nothing
+ * overlaps, is small. While chunk c is computed, chunk c+1 is copied to the
+ * device and chunk c-1's results back to the host, on three streams owned by
+ * the library, with two device copies of every chunk buffer (in
+ * `workspace`). The results are those of the device entry points on the whole
+ * tensors, bit for bit.
  * Host pointers: Q, K, V bf16 [B,H,N,d]; O [B,H,N,d] of type o_dtype; cnt
  *          int32 [B,H,n_q] and idx int32 [B,H,n_q,n_k] (each may be NULL: not
  *          copied back). They must be page-locked (cudaHostAlloc or

@@ -31,7 +31,9 @@
 // warp 9 holds the tcgen05 issuer thread, warps 0-7 compute the elementwise
 // step, two warpgroups taking half of a tile's columns each (a warp reads the
 // TMEM lane quarter warp % 4). TMEM (512 columns):
-//   dQ kernel:   S [0,128), dP [128,256), dQ [256,256+d);
+//   dQ kernel:   S double-buffered [0,128) and [128,256), dP [256,384),
+//                dQ [384,384+d): the products of tile t+1 run while the compute
+//                warps turn tile t's S and dP (already in registers) into dS;
 //   dK/dV kernel: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512).
 #pragma once
 
@@ -65,7 +67,8 @@ constexpr float LOG2E = 1.4426950408889634f;
 
 enum WaitSite : unsigned int {
     W_Q_FULL = 0xD001, W_Q_EMPTY = 0xD002, W_CH_FULL = 0xD003, W_CH_EMPTY = 0xD004, W_S_FULL = 0xD005,
-    W_P_FULL = 0xD006, W_O_FULL = 0xD007, W_ACC_FREE = 0xD008, W_KV_FULL = 0xD009, W_KV_EMPTY = 0xD00A
+    W_P_FULL = 0xD006, W_O_FULL = 0xD007, W_ACC_FREE = 0xD008, W_KV_FULL = 0xD009, W_KV_EMPTY = 0xD00A,
+    W_LOADED = 0xD00B
 };
 
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -269,6 +272,8 @@ struct Ctrl {
     uint64_t kv_full, kv_empty;    // dK/dV kernel: K and V tiles of an item
     uint64_t qs_full[2], qs_empty[2];
     uint64_t s_full, p_full, o_full, acc_free, drain;
+    uint64_t loaded;               // dQ kernel: the compute warps hold S and dP of a tile in registers
+    uint64_t vch_full[2], vch_empty[2];   // dQ kernel: the V ring (the K ring uses ch_full/ch_empty)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -277,12 +282,16 @@ struct Ctrl {
 template <int D, int BQ>
 struct DQLayout {
     static constexpr int SLABS = D / 64;
-    static constexpr int TILE_BYTES = MROWS * D * 2;   // Q, dO, and each K or V chunk (128 rows)
-    static constexpr int NCH = 4;
+    static constexpr int TILE_BYTES = MROWS * D * 2;   // Q, dO, and each K or V tile (128 rows)
+    // Separate rings: a V tile is free once its dP product is done, a K tile
+    // only after its dQ product; three K slots let K(t+1) land while K(t-1)
+    // and K(t) are still in use.
+    static constexpr int NKS = 3, NVS = 2;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_DO = TILE_BYTES;
-    static constexpr int OFF_CH = 2 * TILE_BYTES;
-    static constexpr int OFF_CTRL = OFF_CH + NCH * TILE_BYTES;
+    static constexpr int OFF_K = 2 * TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + NKS * TILE_BYTES;
+    static constexpr int OFF_CTRL = OFF_V + NVS * TILE_BYTES;
     static constexpr int DYN_BYTES = OFF_CTRL + 512 + 1024;
     static_assert(DYN_BYTES <= 232448, "shared memory budget");
 };
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, const Params prm) {
     using L = DQLayout<D, BQ>;
-    constexpr int NCH = L::NCH;
+    constexpr int NKS = L::NKS, NVS = L::NVS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctrl& C = *reinterpret_cast<Ctrl*>(smem + L::OFF_CTRL);
@@ -304,15 +313,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     if (threadIdx.x == 0) {
         mbar_init(&C.q_full, 1);
         mbar_init(&C.q_empty, 1);
-        for (int c = 0; c < NCH; ++c) {
+        for (int c = 0; c < NKS; ++c) {
             mbar_init(&C.ch_full[c], 1);
             mbar_init(&C.ch_empty[c], 1);
+        }
+        for (int c = 0; c < NVS; ++c) {
+            mbar_init(&C.vch_full[c], 1);
+            mbar_init(&C.vch_empty[c], 1);
         }
         mbar_init(&C.s_full, 1);
         mbar_init(&C.p_full, 8);
         mbar_init(&C.o_full, 1);
         mbar_init(&C.acc_free, 8);
         mbar_init(&C.drain, 1);
+        mbar_init(&C.loaded, 8);
         C.abort_flag = 0;
         fence_mbarrier_init();
         fence_proxy_async_smem();
@@ -344,7 +358,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tma_prefetch_descriptor(&tmV);
                 tma_prefetch_descriptor(&tmdO);
             }
-            int k = 0, kq = 0;
+            int g = 0, kq = 0;     // tiles loaded so far (both rings advance once per tile)
+            int gk = 0, gv = 0;    // K and V copies issued (for the abort drain)
             bool ok = true;
             for (int r = blockIdx.x; ok && r < rows; r += gridDim.x) {
                 const int cnt = count_of(r);
@@ -361,7 +376,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 }
                 ++kq;
                 int window = -1;
-                for (int t = 0; t < nt; ++t) {
+                for (int t = 0; t < nt; ++t, ++g) {
                     const int e0 = 2 * t;
                     if ((e0 & 31) == 0) window = entry_of(r, cnt, e0 + lane);
                     int j0 = __shfl_sync(0xFFFFFFFFu, window, e0 & 31);
@@ -369,85 +384,112 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     // An absent (or skipped) block is read at a row past N: zeros.
                     const int r0 = (j0 >= 0 ? j0 : n_k) * BK;
                     const int r1 = (j1 >= 0 ? j1 : n_k) * BK;
-#pragma unroll
-                    for (int kv = 0; kv < 2; ++kv) {   // K(t), then V(t)
-                        const int c = k % NCH;
-                        if (k >= NCH && !wait_warp(&C.ch_empty[c], ((k / NCH) - 1) & 1, abort_flag, W_CH_EMPTY, lim)) {
-                            ok = false;
-                            break;
-                        }
-                        if (lane == 0) {
-                            const CUtensorMap* map = kv ? &tmV : &tmK;
-                            uint8_t* dst = smem + L::OFF_CH + c * L::TILE_BYTES;
-                            mbar_arrive_expect_tx(&C.ch_full[c], L::TILE_BYTES);
-                            for (int sl = 0; sl < L::SLABS; ++sl) {
-                                uint8_t* base = dst + sl * (TILE_N * 128);
-                                tma_load_3d(base, map, &C.ch_full[c], sl * 64, r0, bh);
-                                tma_load_3d(base + BK * 128, map, &C.ch_full[c], sl * 64, r1, bh);
-                            }
-                        }
-                        ++k;
+                    const int ck = g % NKS, cv = g % NVS;
+                    if (g >= NKS && !wait_warp(&C.ch_empty[ck], ((g / NKS) - 1) & 1, abort_flag, W_CH_EMPTY, lim)) {
+                        ok = false;
+                        break;
                     }
-                    if (!ok) break;
+                    if (lane == 0) {
+                        uint8_t* dst = smem + L::OFF_K + ck * L::TILE_BYTES;
+                        mbar_arrive_expect_tx(&C.ch_full[ck], L::TILE_BYTES);
+                        for (int sl = 0; sl < L::SLABS; ++sl) {
+                            tma_load_3d(dst + sl * (TILE_N * 128), &tmK, &C.ch_full[ck], sl * 64, r0, bh);
+                            tma_load_3d(dst + sl * (TILE_N * 128) + BK * 128, &tmK, &C.ch_full[ck], sl * 64, r1, bh);
+                        }
+                    }
+                    gk = g + 1;
+                    if (g >= NVS && !wait_warp(&C.vch_empty[cv], ((g / NVS) - 1) & 1, abort_flag, W_CH_EMPTY, lim)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        uint8_t* dst = smem + L::OFF_V + cv * L::TILE_BYTES;
+                        mbar_arrive_expect_tx(&C.vch_full[cv], L::TILE_BYTES);
+                        for (int sl = 0; sl < L::SLABS; ++sl) {
+                            tma_load_3d(dst + sl * (TILE_N * 128), &tmV, &C.vch_full[cv], sl * 64, r0, bh);
+                            tma_load_3d(dst + sl * (TILE_N * 128) + BK * 128, &tmV, &C.vch_full[cv], sl * 64, r1, bh);
+                        }
+                    }
+                    gv = g + 1;
                 }
             }
             if (*abort_flag && lane == 0) {
+                // Every copy issued must land before the CTA's shared memory is released.
                 if (kq > 0) drain_wait(&C.q_full, (kq - 1) & 1, lim);
-                for (int kk = (k > NCH ? k - NCH : 0); kk < k; ++kk) drain_wait(&C.ch_full[kk % NCH], (kk / NCH) & 1, lim);
+                for (int gg = (gk > NKS ? gk - NKS : 0); gg < gk; ++gg) drain_wait(&C.ch_full[gg % NKS], (gg / NKS) & 1, lim);
+                for (int gg = (gv > NVS ? gv - NVS : 0); gg < gv; ++gg) drain_wait(&C.vch_full[gg % NVS], (gg / NVS) & 1, lim);
             }
         } else if (warp == MMA_WARP && lane == 0) {
             constexpr uint32_t IDESC_S = make_idesc_bf16(MROWS, TILE_N, false);
             constexpr uint32_t IDESC_DQ = make_idesc_bf16(MROWS, D, true);
             const Desc q_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_Q)));
             const Desc do_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_DO)));
-            const Desc ch_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_CH)));
-            const Desc ch_mn = desc_split(mnmajor_desc(smem_u32(smem + L::OFF_CH), TILE_N * 128));
-            const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-            int k = 0, g = 0, kq = 0, rown = 0;
+            const Desc k_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_K)));
+            const Desc v_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_V)));
+            const Desc k_mn = desc_split(mnmajor_desc(smem_u32(smem + L::OFF_K), TILE_N * 128));
+            // S is double-buffered: the products of tile g + 1 go out as soon as the
+            // compute warps have read tile g's S and dP into registers.
+            const uint32_t tSb[2] = {tmem, tmem + 128};
+            const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
+            int g = 0, kq = 0, rown = 0;
             bool ok = true;
-            // S or dP (into d) = A (128 rows, K-major) times B^T (chunk c, K-major).
-            auto issue_sk = [&](uint32_t d, Desc a, int c) {
-                const uint32_t coff = (uint32_t)(c * L::TILE_BYTES) >> 4;
+            // S or dP (into d) = A (128 rows, K-major) times B^T (a ring slot, K-major).
+            auto issue_sk = [&](uint32_t d, Desc a, Desc b, int slot) {
+                const uint32_t coff = (uint32_t)(slot * L::TILE_BYTES) >> 4;
 #pragma unroll
                 for (int sl = 0; sl < L::SLABS; ++sl)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint32_t o = (sl * (MROWS * 128) + kk * 32) >> 4;
-                        umma_ss(d, desc_at(a, o), desc_at(ch_desc, coff + o), IDESC_S, (sl | kk) ? 1u : 0u);
+                        umma_ss(d, desc_at(a, o), desc_at(b, coff + o), IDESC_S, (sl | kk) ? 1u : 0u);
                     }
+            };
+            // The products of tile gt (K in ring slot gt % NKS, V in gt % NVS), into S buffer gt & 1.
+            auto issue_products = [&](int gt) -> bool {
+                const int ck = gt % NKS, cv = gt % NVS;
+                if (!mbar_wait_spin(&C.ch_full[ck], (gt / NKS) & 1, abort_flag, W_CH_FULL, lim) ||
+                    !mbar_wait_spin(&C.vch_full[cv], (gt / NVS) & 1, abort_flag, W_CH_FULL, lim))
+                    return false;
+                tc_fence_after();
+                issue_sk(tSb[gt & 1], q_desc, k_desc, ck);
+                issue_sk(tdP, do_desc, v_desc, cv);
+                umma_commit(&C.s_full);
+                umma_commit(&C.vch_empty[cv]);          // V is no longer needed
+                return true;
             };
             for (int r = blockIdx.x; ok && r < rows; r += gridDim.x) {
                 const int nt = (count_of(r) + 1) / 2;
                 if (nt == 0) continue;
                 if (!mbar_wait_spin(&C.q_full, kq & 1, abort_flag, W_Q_FULL, lim)) { ok = false; break; }
                 ++kq;
+                // The first tile's dP overwrites the previous tile's, which the
+                // compute warps must have read.
+                if (g > 0 && !mbar_wait_spin(&C.loaded, (g - 1) & 1, abort_flag, W_LOADED, lim)) { ok = false; break; }
+                if (!issue_products(g)) { ok = false; break; }
+                if (nt == 1) umma_commit(&C.q_empty);
                 for (int t = 0; t < nt; ++t) {
-                    const int ck = k % NCH, cv = (k + 1) % NCH;
-                    if (!mbar_wait_spin(&C.ch_full[ck], (k / NCH) & 1, abort_flag, W_CH_FULL, lim) ||
-                        !mbar_wait_spin(&C.ch_full[cv], ((k + 1) / NCH) & 1, abort_flag, W_CH_FULL, lim)) {
-                        ok = false;
-                        break;
+                    if (t + 1 < nt) {
+                        if (!mbar_wait_spin(&C.loaded, g & 1, abort_flag, W_LOADED, lim) ||
+                            !issue_products(g + 1)) {
+                            ok = false;
+                            break;
+                        }
+                        if (t + 2 == nt) umma_commit(&C.q_empty);
                     }
-                    tc_fence_after();
-                    issue_sk(tS, q_desc, ck);
-                    issue_sk(tdP, do_desc, cv);
-                    umma_commit(&C.s_full);
-                    umma_commit(&C.ch_empty[cv]);          // V(t) is no longer needed
-                    if (t + 1 == nt) umma_commit(&C.q_empty);
                     if (!mbar_wait_spin(&C.p_full, g & 1, abort_flag, W_P_FULL, lim)) { ok = false; break; }
                     if (t == 0 && rown > 0 && !mbar_wait_spin(&C.acc_free, (rown - 1) & 1, abort_flag, W_ACC_FREE, lim)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const int ck = g % NKS;
                     uint64_t bk[TILE_N / 16];
                     const uint32_t coff = (uint32_t)(ck * L::TILE_BYTES) >> 4;
 #pragma unroll
-                    for (int kk = 0; kk < TILE_N / 16; ++kk) bk[kk] = desc_at(ch_mn, coff + ((kk * 16 * 128) >> 4));
-                    umma_ts_halves<TILE_N / 16>(tdQ, tS, tS + 64, bk, IDESC_DQ, t > 0 ? 1u : 0u);
-                    umma_commit(&C.ch_empty[ck]);
+                    for (int kk = 0; kk < TILE_N / 16; ++kk) bk[kk] = desc_at(k_mn, coff + ((kk * 16 * 128) >> 4));
+                    umma_ts_halves<TILE_N / 16>(tdQ, tSb[g & 1], tSb[g & 1] + 64, bk, IDESC_DQ, t > 0 ? 1u : 0u);
+                    umma_commit(&C.ch_empty[ck]);          // K is no longer needed
                     if (t + 1 == nt) umma_commit(&C.o_full);
-                    k += 2;
                     ++g;
                 }
                 ++rown;
@@ -463,7 +505,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int wq = warp & 3;                 // TMEM lane quarter
         const int row = wq * 32 + lane;          // query row within the tile
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_off, tdP = tmem + 128 + lane_off, tdQ = tmem + 256 + lane_off;
+        const uint32_t tSb[2] = {tmem + lane_off, tmem + 128 + lane_off};
+        const uint32_t tdP = tmem + 256 + lane_off, tdQ = tmem + 384 + lane_off;
         const float sl2 = prm.scale_log2;
         const bool f32 = prm.out_f32 != 0;
         int g = 0, rown = 0;
@@ -497,16 +540,21 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int nvalid = j < 0 ? 0 : min(BK, prm.N - j * BK);
                 if (!wait_warp(&C.s_full, g & 1, abort_flag, W_S_FULL, lim)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t tS = tSb[g & 1];
+                uint32_t s[64], dp[64];
+                tmem_ld64(tS + wg * 64, s);
+                tmem_ld64(tdP + wg * 64, dp);
+                // S and dP are in registers: the next tile's products may overwrite dP.
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&C.loaded);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {   // two chunks of 32 keys
-                    const int col = wg * 64 + h * 32;
-                    uint32_t s[32], dp[32];
-                    tmem_ld32(tS + col, s);
-                    tmem_ld32(tdP + col, dp);
                     const int nv = nvalid - h * 32;
                     const uint32_t vm = nv >= 32 ? 0xFFFFFFFFu : (nv <= 0 ? 0u : ((1u << nv) - 1u));
                     uint32_t pk[16], dk[16];
-                    p_ds_chunk(s, dp, l2, dv, vm, sl2, pk, dk);
+                    p_ds_chunk(*reinterpret_cast<const uint32_t(*)[32]>(s + 32 * h),
+                               *reinterpret_cast<const uint32_t(*)[32]>(dp + 32 * h), l2, dv, vm, sl2, pk, dk);
                     // dS goes over this warpgroup's own S columns (already read).
                     tmem_st16_nowait(tS + wg * 64 + h * 16, dk);
                 }

@@ -95,26 +95,18 @@ int topk_count(double k, int n_k) {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Mask workspace. Rows of up to FM_MAX_NK key blocks go through the
-// one-launch kernel (pooled means and its work counters); longer rows through
-// the three-kernel path (pooled means and the logit matrix).
 struct Workspace {
-    size_t qbar, kbar, logits, counters, total;
+    size_t qbar, kbar, logits, total;
     int ld;
-    bool fused;
 };
 
 Workspace workspace_layout(const Dims& g) {
     Workspace w;
-    w.fused = g.n_k <= sa::mask::FM_MAX_NK;
     w.ld = (g.n_k + 3) & ~3;
     w.qbar = 0;
     w.kbar = round256((size_t)g.BH * g.n_q * g.d * sizeof(float));
-    w.logits = w.counters = w.kbar + round256((size_t)g.BH * g.n_k * g.d * sizeof(float));
-    if (w.fused)
-        w.total = w.counters + round256((size_t)(1 + g.BH) * sizeof(int));
-    else
-        w.total = w.logits + round256((size_t)g.BH * g.n_q * w.ld * sizeof(float));
+    w.logits = w.kbar + round256((size_t)g.BH * g.n_k * g.d * sizeof(float));
+    w.total = w.logits + round256((size_t)g.BH * g.n_q * w.ld * sizeof(float));
     return w;
 }
 
@@ -172,19 +164,6 @@ sa_status make_map_u8(CUtensorMap* map, const void* base, const Dims& g, int row
 }
 
 // ------------------------------------------------------------ launches
-// Multiprocessor count of the current device (cached per device).
-int sm_count() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
-
 template <int D>
 sa_status launch_pool_score(const Dims& g, const void* Q, const void* K, const Workspace& w,
                             uint8_t* ws, cudaStream_t st) {
@@ -205,52 +184,6 @@ sa_status launch_pool_score(const Dims& g, const void* Q, const void* K, const W
     return cuda_check(cudaGetLastError(), "score_kernel launch");
 }
 
-template <int D>
-sa_status launch_fused_mask(const Dims& g, const void* Q, const void* K, double k, double p, int32_t* cnt,
-                            int32_t* idx, uint8_t* mask, float* P_out, const Workspace& w, uint8_t* ws,
-                            cudaStream_t st) {
-    namespace M = sa::mask;
-    M::FusedMaskParams prm;
-    prm.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
-    prm.K = reinterpret_cast<const __nv_bfloat16*>(K);
-    prm.Qbar = reinterpret_cast<float*>(ws + w.qbar);
-    prm.Kbar = reinterpret_cast<float*>(ws + w.kbar);
-    prm.counters = reinterpret_cast<int*>(ws + w.counters);
-    prm.cnt = cnt;
-    prm.idx = idx;
-    prm.mask = mask;
-    prm.P_out = P_out;
-    prm.N = g.N;
-    prm.bq = g.bq;
-    prm.bk = g.bk;
-    prm.n_q = g.n_q;
-    prm.n_k = g.n_k;
-    prm.BH = g.BH;
-    prm.kc = topk_count(k, g.n_k);
-    prm.p = p;
-    prm.scale = (float)(1.0 / std::sqrt((double)D));
-    prm.pool_items = (g.n_q + g.n_k + M::FM_POOL_GROUP - 1) / M::FM_POOL_GROUP;
-    const int R = M::fm_rows_per_item(g.n_k);
-    prm.sel_items = (g.n_q + R - 1) / R;
-    prm.total_items = g.BH * (prm.pool_items + prm.sel_items);
-    prm.wait_limit_ns = WAIT_LIMIT_NS;
-    const size_t smem = M::fm_smem_bytes<D>(g.n_k);
-    auto kern = M::fused_mask_kernel<D>;
-    sa_status s;
-    if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
-                        "fused_mask_kernel shared-memory attribute")) != SA_OK)
-        return s;
-    // The work counters start at zero on every launch.
-    if ((s = cuda_check(cudaMemsetAsync(prm.counters, 0, (size_t)(1 + g.BH) * sizeof(int), st),
-                        "clear the mask work counters")) != SA_OK)
-        return s;
-    const int per_sm = smem <= 110 * 1024 ? 2 : 1;
-    int grid = sm_count() * per_sm;
-    if (grid > prm.total_items) grid = prm.total_items;
-    kern<<<grid, M::FM_THREADS, smem, st>>>(prm);
-    return cuda_check(cudaGetLastError(), "fused_mask_kernel launch");
-}
-
 template <bool FROM_LOGITS>
 sa_status launch_select(const Dims& g, const float* in, int ld_in, double k, double p, int32_t* cnt,
                         int32_t* idx, uint8_t* mask, float* P_out, cudaStream_t st) {
@@ -269,6 +202,18 @@ sa_status launch_select(const Dims& g, const float* in, int ld_in, double k, dou
     return cuda_check(cudaGetLastError(), "select_kernel launch");
 }
 
+// Multiprocessor count of the current device (cached per device).
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 // Knobs of the failure-detection test hook; normal launches use the defaults.
 struct AttnTestKnobs {
@@ -525,12 +470,6 @@ sa_status sparse_attn_mask(const sa_shape* shape, const void* Q, const void* K, 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const Workspace w = workspace_layout(g);
     uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
-    if (w.fused) {
-        s = (g.d == 128) ? launch_fused_mask<128>(g, Q, K, k, p, cnt, idx, mask_or_null, P_out_or_null, w, ws, st)
-                         : launch_fused_mask<64>(g, Q, K, k, p, cnt, idx, mask_or_null, P_out_or_null, w, ws, st);
-        if (s != SA_OK) return s;
-        return ok();
-    }
     s = (g.d == 128) ? launch_pool_score<128>(g, Q, K, w, ws, st) : launch_pool_score<64>(g, Q, K, w, ws, st);
     if (s != SA_OK) return s;
     s = launch_select<true>(g, reinterpret_cast<const float*>(ws + w.logits), w.ld, k, p, cnt, idx,

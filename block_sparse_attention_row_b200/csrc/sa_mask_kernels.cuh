@@ -282,11 +282,20 @@ __device__ Boundary boundary_search(const uint32_t* __restrict__ bits, const uin
     return {v, n_above, mass_above};
 }
 
-// The selection of one score row by one warp (all 32 lanes): `bits` holds the
-// row's n_k scores as fp32 bit patterns (in [0, 1]), `masses` room for n_k
-// fixed-point masses (written here when p > 0). The kept set is the first L
-// entries of the order "score descending, then index ascending", L =
-// max(kc, m_p):
+constexpr int SEL_MAX_WARPS = 4;
+constexpr int SEL_SMEM_BUDGET = 200 * 1024;
+
+// Warps (rows) per CTA of select_kernel for a row length n_k: each warp
+// holds its row's score bits and fixed-point masses in shared memory (12
+// bytes per entry, rounded up to keep the masses 8-byte aligned).
+__host__ __device__ inline int select_row_bytes(int n_k) { return 4 * ((n_k + 1) & ~1) + 8 * n_k; }
+inline int select_warps_per_cta(int n_k) {
+    int w = SEL_SMEM_BUDGET / select_row_bytes(n_k);
+    return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : w);
+}
+
+// One warp per score row. The kept set is the first L entries of the order
+// "score descending, then index ascending", L = max(kc, m_p):
 //   kc  = number of Top-k blocks (computed on the host);
 //   m_p = shortest prefix whose fixed-point mass reaches T = ceil(p * W).
 // m_p comes from the mass boundary v (entries above v, then as many of the
@@ -294,10 +303,55 @@ __device__ Boundary boundary_search(const uint32_t* __restrict__ bits, const uin
 // count boundary of kc is searched the same way. The kept indices are then
 // written in ascending order, ties at the boundary taken by lower index.
 // The result equals the prefix of a full sort bit for bit.
-__device__ __forceinline__ void select_row_warp(const uint32_t* __restrict__ bits, uint64_t* __restrict__ masses,
-                                                int n_k, int kc, double p, int32_t* __restrict__ idx_row,
-                                                uint8_t* __restrict__ mask_row, int32_t* __restrict__ cnt_out,
-                                                int lane) {
+template <bool FROM_LOGITS>
+__global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
+select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
+              int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
+              float* __restrict__ P_out) {
+    extern __shared__ __align__(8) unsigned char sel_smem[];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int wpc = blockDim.x / 32;
+    const long long row = (long long)blockIdx.x * wpc + warp;
+    if (row >= n_rows) return;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(sel_smem + (size_t)warp * select_row_bytes(n_k));
+    uint64_t* masses = reinterpret_cast<uint64_t*>(bits + ((n_k + 1) & ~1));
+    const float* src = in + (size_t)row * ld_in;
+
+    if (FROM_LOGITS) {
+        float mx = -INFINITY;
+        for (int j = lane; j < n_k; j += 32) mx = fmaxf(mx, src[j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        // exp(x - max) as 2^((x - max) log2 e) on the MUFU unit (relative error
+        // about 2e-7, far below the 1e-6 near-tie scale), and one reciprocal of
+        // the sum; P is clamped to 1 so its fixed-point mass stays <= 2^31.
+        const float mxl = mx * 1.4426950408889634f;
+        float sum = 0.f;
+        for (int j = lane; j < n_k; j += 32) {
+            const float e = ex2_approx(fmaf(src[j], 1.4426950408889634f, -mxl));
+            bits[j] = __float_as_uint(e);
+            sum += e;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        const float inv = 1.0f / sum;
+        for (int j = lane; j < n_k; j += 32) {
+            const float pj = fminf(__uint_as_float(bits[j]) * inv, 1.0f);
+            bits[j] = __float_as_uint(pj);
+            if (P_out) P_out[(size_t)row * n_k + j] = pj;
+        }
+    } else {
+        bool bad = false;
+        for (int j = lane; j < n_k; j += 32) {
+            const uint32_t b = __float_as_uint(src[j]);
+            bad |= (b > 0x3F800000u);  // negative, > 1, Inf or NaN
+            bits[j] = b;
+        }
+        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0)
+            record_error(SA_STATUS_DEVICE_ASSERT, 0x5E1Eu);
+    }
+    __syncwarp();
+
     // L = number of kept entries; (v, n_above) = its boundary score and the
     // number of entries strictly above it.
     int L = kc;
@@ -329,6 +383,8 @@ __device__ __forceinline__ void select_row_warp(const uint32_t* __restrict__ bit
     }
     L = min(L, n_k);
 
+    int32_t* idx_row = idx + (size_t)row * n_k;
+    uint8_t* mask_row = mask ? mask + (size_t)row * n_k : nullptr;
     if (L == n_k) {
         for (int j = lane; j < n_k; j += 32) {
             idx_row[j] = j;
@@ -360,336 +416,7 @@ __device__ __forceinline__ void select_row_warp(const uint32_t* __restrict__ bit
             kept_before += __popc(keep_ballot);
         }
     }
-    if (lane == 0) *cnt_out = L;
-}
-
-// Row softmax of n_k logits by one warp, into `bits` (fp32 bit patterns of
-// P, in [0, 1]) and, if P_row is set, into global memory. exp(x - max) is
-// 2^((x - max) log2 e) on the MUFU unit (relative error about 2e-7, far below
-// the 1e-6 near-tie scale), with one reciprocal of the sum; P is clamped to 1
-// so its fixed-point mass stays <= 2^31. `src` and `bits` may be the same
-// array (each entry is read before it is overwritten, by the same lane).
-__device__ __forceinline__ void softmax_row_warp(const float* src, uint32_t* bits, int n_k, float* P_row,
-                                                 int lane) {
-    float mx = -INFINITY;
-    for (int j = lane; j < n_k; j += 32) mx = fmaxf(mx, src[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    const float mxl = mx * 1.4426950408889634f;
-    float sum = 0.f;
-    for (int j = lane; j < n_k; j += 32) {
-        const float e = ex2_approx(fmaf(src[j], 1.4426950408889634f, -mxl));
-        bits[j] = __float_as_uint(e);
-        sum += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-    const float inv = 1.0f / sum;
-    for (int j = lane; j < n_k; j += 32) {
-        const float pj = fminf(__uint_as_float(bits[j]) * inv, 1.0f);
-        bits[j] = __float_as_uint(pj);
-        if (P_row) P_row[j] = pj;
-    }
-}
-
-constexpr int SEL_MAX_WARPS = 4;
-constexpr int SEL_SMEM_BUDGET = 200 * 1024;
-
-// Warps (rows) per CTA of select_kernel for a row length n_k: each warp
-// holds its row's score bits and fixed-point masses in shared memory (12
-// bytes per entry, rounded up to keep the masses 8-byte aligned).
-__host__ __device__ inline int select_row_bytes(int n_k) { return 4 * ((n_k + 1) & ~1) + 8 * n_k; }
-inline int select_warps_per_cta(int n_k) {
-    int w = SEL_SMEM_BUDGET / select_row_bytes(n_k);
-    return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : w);
-}
-
-// One warp per score row: the row's softmax (from logits) or the given P,
-// then select_row_warp.
-template <bool FROM_LOGITS>
-__global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
-select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
-              int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
-              float* __restrict__ P_out) {
-    extern __shared__ __align__(8) unsigned char sel_smem[];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int wpc = blockDim.x / 32;
-    const long long row = (long long)blockIdx.x * wpc + warp;
-    if (row >= n_rows) return;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(sel_smem + (size_t)warp * select_row_bytes(n_k));
-    uint64_t* masses = reinterpret_cast<uint64_t*>(bits + ((n_k + 1) & ~1));
-    const float* src = in + (size_t)row * ld_in;
-
-    if (FROM_LOGITS) {
-        softmax_row_warp(src, bits, n_k, P_out ? P_out + (size_t)row * n_k : nullptr, lane);
-    } else {
-        bool bad = false;
-        for (int j = lane; j < n_k; j += 32) {
-            const uint32_t b = __float_as_uint(src[j]);
-            bad |= (b > 0x3F800000u);  // negative, > 1, Inf or NaN
-            bits[j] = b;
-        }
-        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0)
-            record_error(SA_STATUS_DEVICE_ASSERT, 0x5E1Eu);
-    }
-    __syncwarp();
-    select_row_warp(bits, masses, n_k, kc, p, idx + (size_t)row * n_k, mask ? mask + (size_t)row * n_k : nullptr,
-                    cnt + row, lane);
-}
-
-}  // namespace mask
-}  // namespace sa
-
-namespace sa {
-namespace mask {
-
-// ------------------------------------------------------------ one launch
-// Steps 1-3 in a single persistent kernel. Work items are taken from a
-// device-side counter in one global order, head by head with a lag of one:
-//   pool(0), pool(1) select(0), pool(2) select(1), ..., select(BH-1)
-// where pool(h) is the pooling of head h's query and key blocks (groups of
-// FM_POOL_GROUP blocks per item) and select(h) the scoring, softmax and
-// selection of head h's rows (FM rows per item). A select item waits for its
-// head's pooled-block count to be complete; every pool item it waits for was
-// claimed earlier by a running CTA and never waits itself, so the order
-// cannot deadlock, whatever the number of resident CTAs. The HBM-bound
-// pooling of head h+1 then runs while other CTAs score and select head h.
-constexpr int FM_THREADS = 256;
-constexpr int FM_MAX_NK = 1280;     // longer rows use the three-kernel path
-constexpr int FM_POOL_GROUP = 8;    // blocks per pool item
-constexpr int FM_KCHUNK = 64;       // key blocks per staged chunk of Kbar
-constexpr unsigned int FM_WAIT_SITE = 0xF001;
-
-__host__ __device__ inline int fm_rows_per_item(int n_k) { return n_k <= 640 ? 32 : 16; }
-__host__ __device__ inline int fm_ld(int n_k) { return (n_k + 1) & ~1; }
-
-struct FusedMaskParams {
-    const __nv_bfloat16* Q;
-    const __nv_bfloat16* K;
-    float* Qbar;      // [BH, n_q, d]
-    float* Kbar;      // [BH, n_k, d]
-    int* counters;    // [0]: next work item; [1 + bh]: pooled blocks of head bh (zero at launch)
-    int32_t* cnt;
-    int32_t* idx;
-    uint8_t* mask;
-    float* P_out;
-    int N, bq, bk, n_q, n_k, BH, kc;
-    double p;
-    float scale;
-    int pool_items, sel_items, total_items;   // per head, per head, in all
-    unsigned long long wait_limit_ns;
-};
-
-// Shared-memory bytes of the one-launch kernel for a row length n_k.
-template <int D>
-__host__ __device__ inline size_t fm_smem_bytes(int n_k) {
-    const int R = fm_rows_per_item(n_k);
-    return (size_t)D * R * 4                       // Qbar rows, channel-major
-           + (size_t)D * FM_KCHUNK * 4             // a chunk of Kbar, channel-major
-           + (size_t)R * fm_ld(n_k) * 4            // logits, then P bits, per row
-           + (size_t)(FM_THREADS / 32) * n_k * 8   // fixed-point masses, per warp
-           + (size_t)2 * (POOL_THREADS / (D / 8)) * D * 4   // pool partial sums, two blocks at a time
-           + 16;
-}
-
-// Mean of the valid tokens of one block, by 128 threads (t = 0..127), with
-// the same decomposition and summation order as pool_kernel.
-template <int D>
-__device__ __forceinline__ void pool_block(const __nv_bfloat16* __restrict__ X, float* __restrict__ out, int valid,
-                                           float* red, int t) {
-    constexpr int CG = D / 8;
-    constexpr int RG = POOL_THREADS / CG;
-    const uint4* src = reinterpret_cast<const uint4*>(X);
-    const int cg = t % CG, rg = t / CG;
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 8
-    for (int r = rg; r < valid; r += RG) {
-        const uint4 v = __ldg(src + (size_t)r * CG + cg);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            acc[2 * e] += __uint_as_float(w[e] << 16);
-            acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[rg * D + cg * 8 + e] = acc[e];
-}
-
-template <int D>
-__device__ __forceinline__ void pool_block_finish(float* __restrict__ out, int valid, const float* red, int t) {
-    constexpr int RG = POOL_THREADS / (D / 8);
-    for (int c = t; c < D; c += POOL_THREADS) {
-        float s = 0.f;
-#pragma unroll
-        for (int g = 0; g < RG; ++g) s += red[g * D + c];
-        out[c] = s / (float)valid;
-    }
-}
-
-template <int D>
-__global__ void __launch_bounds__(FM_THREADS, 1)
-fused_mask_kernel(const FusedMaskParams prm) {
-    constexpr int RG = POOL_THREADS / (D / 8);
-    extern __shared__ __align__(16) unsigned char fm_smem[];
-    const int n_k = prm.n_k, n_q = prm.n_q;
-    const int R = fm_rows_per_item(n_k);
-    const int ld = fm_ld(n_k);
-    float* qs = reinterpret_cast<float*>(fm_smem);                 // [D][R]
-    float* ks = qs + D * R;                                          // [D][FM_KCHUNK]
-    float* logits = ks + D * FM_KCHUNK;                              // [R][ld]
-    uint64_t* masses = reinterpret_cast<uint64_t*>(logits + (size_t)R * ld);   // [8][n_k]
-    float* red = reinterpret_cast<float*>(masses + (size_t)(FM_THREADS / 32) * n_k);   // [2][RG][D]
-    int* item_slot = reinterpret_cast<int*>(red + 2 * RG * D);
-    const int t = threadIdx.x, warp = t / 32, lane = t % 32;
-    const int per_seg = prm.pool_items + prm.sel_items;
-
-    for (;;) {
-        if (t == 0) *item_slot = atomicAdd(prm.counters, 1);
-        __syncthreads();
-        const int x = *item_slot;
-        __syncthreads();
-        if (x >= prm.total_items) break;
-        // Decode: segment 0 = pool(0); segment m in [1, BH) = pool(m) then
-        // select(m-1); segment BH = select(BH-1).
-        int bh, off;
-        bool is_pool;
-        if (x < prm.pool_items) {
-            bh = 0, off = x, is_pool = true;
-        } else {
-            const int y = x - prm.pool_items;
-            const int m = y / per_seg + 1;
-            off = y % per_seg;
-            if (m < prm.BH && off < prm.pool_items) {
-                bh = m, is_pool = true;
-            } else {
-                bh = m - 1, is_pool = false;
-                if (m < prm.BH) off -= prm.pool_items;
-            }
-        }
-        if (is_pool) {
-            // ---------------------------------------------- pool item
-            const int nblk = n_q + n_k;
-            const int b0 = off * FM_POOL_GROUP;
-            const int b1 = min(nblk, b0 + FM_POOL_GROUP);
-            const int half = t / 128, th = t % 128;
-            float* rh = red + half * RG * D;
-            for (int b = b0 + half; b - half < b1; b += 2) {
-                const bool active = b < b1;
-                const bool isq = b < n_q;
-                const int blk = isq ? b : b - n_q;
-                const int bs = isq ? prm.bq : prm.bk;
-                const int lo = blk * bs;
-                const int valid = active ? min(prm.N - lo, bs) : 0;
-                const __nv_bfloat16* X = (isq ? prm.Q : prm.K) + ((size_t)bh * prm.N + lo) * D;
-                float* out = isq ? prm.Qbar + ((size_t)bh * n_q + blk) * D : prm.Kbar + ((size_t)bh * n_k + blk) * D;
-                if (active) pool_block<D>(X, out, valid, rh, th);
-                __syncthreads();
-                if (active) pool_block_finish<D>(out, valid, rh, th);
-                __syncthreads();
-            }
-            __threadfence();
-            __syncthreads();
-            if (t == 0) atomicAdd(prm.counters + 1 + bh, b1 - b0);
-        } else {
-            // -------------------------------------------- select item
-            const int r0 = off * R;
-            const int nr = min(R, n_q - r0);
-            if (t == 0) {
-                const int need = n_q + n_k;
-                volatile int* done = prm.counters + 1 + bh;
-                bool ok = *done >= need;
-                if (!ok) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (!(ok = (*done >= need))) {
-                        __nanosleep(256);
-                        if (globaltimer_ns() - t0 > prm.wait_limit_ns) break;
-                    }
-                }
-                if (!ok) record_error(SA_STATUS_TIMEOUT, FM_WAIT_SITE);
-                *item_slot = ok ? 1 : 0;
-            }
-            __syncthreads();
-            const bool ready = *item_slot != 0;
-            __syncthreads();
-            if (!ready) continue;
-            __threadfence();
-            // Qbar rows of the item, channel-major (rows past nr are zero).
-            const float* qsrc = prm.Qbar + ((size_t)bh * n_q + r0) * D;
-            for (int e = t; e < R * (D / 4); e += FM_THREADS) {
-                const int r = e % R, c4 = e / R;
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (r < nr) v = __ldcg(reinterpret_cast<const float4*>(qsrc + (size_t)r * D) + c4);
-                qs[(4 * c4 + 0) * R + r] = v.x;
-                qs[(4 * c4 + 1) * R + r] = v.y;
-                qs[(4 * c4 + 2) * R + r] = v.z;
-                qs[(4 * c4 + 3) * R + r] = v.w;
-            }
-            const float* ksrc = prm.Kbar + (size_t)bh * n_k * D;
-            const int kk = t % FM_KCHUNK, rgp = t / FM_KCHUNK;   // key in chunk, row group (4 groups)
-            const int rpt = R / 4;                                   // rows per thread: 8 or 4
-            for (int j0 = 0; j0 < n_k; j0 += FM_KCHUNK) {
-                __syncthreads();   // the previous chunk is consumed (and qs is written)
-                for (int e = t; e < FM_KCHUNK * (D / 4); e += FM_THREADS) {
-                    const int jj = e % FM_KCHUNK, c4 = e / FM_KCHUNK;
-                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (j0 + jj < n_k) v = __ldcg(reinterpret_cast<const float4*>(ksrc + (size_t)(j0 + jj) * D) + c4);
-                    ks[(4 * c4 + 0) * FM_KCHUNK + jj] = v.x;
-                    ks[(4 * c4 + 1) * FM_KCHUNK + jj] = v.y;
-                    ks[(4 * c4 + 2) * FM_KCHUNK + jj] = v.z;
-                    ks[(4 * c4 + 3) * FM_KCHUNK + jj] = v.w;
-                }
-                __syncthreads();
-                float acc[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-                if (rpt == 8) {
-#pragma unroll 4
-                    for (int c = 0; c < D; ++c) {
-                        const float kv = ks[c * FM_KCHUNK + kk];
-                        const float4 a = *reinterpret_cast<const float4*>(qs + c * R + rgp * 8);
-                        const float4 b = *reinterpret_cast<const float4*>(qs + c * R + rgp * 8 + 4);
-                        acc[0] = fmaf(a.x, kv, acc[0]);
-                        acc[1] = fmaf(a.y, kv, acc[1]);
-                        acc[2] = fmaf(a.z, kv, acc[2]);
-                        acc[3] = fmaf(a.w, kv, acc[3]);
-                        acc[4] = fmaf(b.x, kv, acc[4]);
-                        acc[5] = fmaf(b.y, kv, acc[5]);
-                        acc[6] = fmaf(b.z, kv, acc[6]);
-                        acc[7] = fmaf(b.w, kv, acc[7]);
-                    }
-                } else {
-#pragma unroll 4
-                    for (int c = 0; c < D; ++c) {
-                        const float kv = ks[c * FM_KCHUNK + kk];
-                        const float4 a = *reinterpret_cast<const float4*>(qs + c * R + rgp * 4);
-                        acc[0] = fmaf(a.x, kv, acc[0]);
-                        acc[1] = fmaf(a.y, kv, acc[1]);
-                        acc[2] = fmaf(a.z, kv, acc[2]);
-                        acc[3] = fmaf(a.w, kv, acc[3]);
-                    }
-                }
-                if (j0 + kk < n_k) {
-                    for (int i = 0; i < rpt; ++i) logits[(size_t)(rgp * rpt + i) * ld + j0 + kk] = acc[i] * prm.scale;
-                }
-            }
-            __syncthreads();
-            // Softmax and selection, one warp per row.
-            uint64_t* wm = masses + (size_t)warp * n_k;
-            for (int r = warp; r < nr; r += FM_THREADS / 32) {
-                const size_t row = (size_t)bh * n_q + r0 + r;
-                uint32_t* bits = reinterpret_cast<uint32_t*>(logits + (size_t)r * ld);
-                softmax_row_warp(logits + (size_t)r * ld, bits, n_k, prm.P_out ? prm.P_out + row * n_k : nullptr, lane);
-                __syncwarp();
-                select_row_warp(bits, wm, n_k, prm.kc, prm.p, prm.idx + row * n_k,
-                                prm.mask ? prm.mask + row * n_k : nullptr, prm.cnt + row, lane);
-                __syncwarp();
-            }
-            __syncthreads();
-        }
-    }
+    if (lane == 0) cnt[row] = L;
 }
 
 }  // namespace mask

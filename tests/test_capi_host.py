@@ -47,26 +47,11 @@ def test_version(lib):
 def test_workspace_bytes(lib, B, H, N, d, bq, bk):
     from block_sparse_attention_row_b200.capi import make_shape
     n_q, n_k = math.ceil(N / bq), math.ceil(N / bk)
-    assert lib.sparse_attn_mask_workspace_bytes(ctypes.byref(make_shape(B, H, N, d, bq, bk))) == \
-        _mask_ws(B * H, n_q, n_k, d)
-
-
-def _mask_ws(BH, n_q, n_k, d):
-    """Pooled means, then the one-launch kernel's work counters (rows of up to
-    1280 key blocks) or the three-kernel path's logit matrix (longer rows)."""
+    ld = (n_k + 3) // 4 * 4
     r = lambda x: (x + 255) // 256 * 256
-    base = r(BH * n_q * d * 4) + r(BH * n_k * d * 4)
-    if n_k <= 1280:
-        return base + r((1 + BH) * 4)
-    return base + r(BH * n_q * ((n_k + 3) // 4 * 4) * 4)
-
-
-def test_workspace_bytes_long_rows_use_the_logit_matrix(lib):
-    from block_sparse_attention_row_b200.capi import make_shape
-    for N in (64 * 1280, 64 * 1281, 64 * 4000):
-        n_q, n_k = -(-N // 128), -(-N // 64)
-        assert lib.sparse_attn_mask_workspace_bytes(ctypes.byref(make_shape(1, 2, N, 128, 128, 64))) == \
-            _mask_ws(2, n_q, n_k, 128)
+    want = r(B * H * n_q * d * 4) + r(B * H * n_k * d * 4) + r(B * H * n_q * ld * 4)
+    sh = make_shape(B, H, N, d, bq, bk)
+    assert lib.sparse_attn_mask_workspace_bytes(ctypes.byref(sh)) == want
 
 
 def test_workspace_bytes_rejects_bad_shapes(lib):
@@ -124,7 +109,8 @@ def test_host_pipeline_workspace_and_validation(lib):
     for hpc, out_dtype, esize in ((0, 0, 2), (3, 0, 2), (7, 1, 4), (40, 0, 2), (100, 0, 2)):
         got = lib.sparse_attn_host_workspace_bytes(ctypes.byref(make_shape(B, H, N, d, 128, 64)), out_dtype, hpc)
         h = min(H, -(-2368 // n_q)) if hpc == 0 else min(hpc, H)
-        mws = _mask_ws(h, n_q, n_k, d)
+        ld = (n_k + 3) // 4 * 4
+        mws = r(h * n_q * d * 4) + r(h * n_k * d * 4) + r(h * n_q * ld * 4)
         per = 3 * r(h * N * d * 2) + r(h * N * d * esize) + r(h * n_q * 4) + r(h * n_q * n_k * 4) + r(mws)
         assert got == 2 * per, (hpc, got, 2 * per)
     good = ctypes.byref(make_shape(1, 2, 4096, 64, 64, 64))

@@ -21,10 +21,9 @@ from block_sparse_attention_row_b200 import capi
 
 
 def test_noalloc_rejects_workspaces_beyond_its_scratch():
-    """Host-side check, no GPU work: the Long layer (40 heads of 75,600 tokens)
-    needs more than 32 MiB."""
+    """Host-side check, no GPU work: the Wan-like layer needs more than 32 MiB."""
     lib = capi.load_library()
-    shape = capi.make_shape(1, 40, 75600, 128, 128, 64)
+    shape = capi.make_shape(1, 40, 32760, 128, 128, 64)
     need = lib.sparse_attn_mask_workspace_bytes(ctypes.byref(shape))
     assert need > capi.NOALLOC_SCRATCH_BYTES
     a = ctypes.c_void_p(256)

@@ -498,6 +498,23 @@ def run_ours(args):
                 qms, f8ms = loop_time([do_q8, do_f8], max(10, min(args.steps, 20)))
                 entry.update({"fp8_quantize_ms": qms, "fp8_fwd_ms": f8ms,
                               "fp8_fwd_kept_tile_tflops": fl_t / (f8ms * 1e-3) / 1e12})
+            if d == 128:
+                # The sparse + linear combination on the same mask (alpha seeded U[0, 1]).
+                from block_sparse_attention_row_b200 import sparse_attn_sparse_linear, sparse_linear_workspace_bytes
+                from synth import make_mix_ratio
+                alpha = make_mix_ratio(B, H, N, seed=cfg.seed + 11, device=dev)
+                lws = torch.empty(sparse_linear_workspace_bytes(B, H, N, d, bq, bk), dtype=torch.uint8, device=dev)
+                Omix = torch.empty_like(O)
+                sparse_attn_fwd(Q, K, V, mo["cnt"], mo["idx"], bq, bk, out=O)
+
+                def do_sl():
+                    sparse_attn_sparse_linear(Q, K, V, mo["cnt"], mo["idx"], O, alpha, bq, bk, out=Omix,
+                                              workspace=lws)
+                for _ in range(2):
+                    do_sl()
+                sl_ms, = loop_time([do_sl], max(5, min(args.steps, 10)))
+                entry.update({"sparse_linear_ms": sl_ms,
+                              "sparse_linear_kept_tile_tflops": fl_t / (sl_ms * 1e-3) / 1e12})
             extra_paths[tag] = entry
         check_device_error(dev)
         # End to end through the public host-buffer entry point (pinned host
@@ -573,7 +590,9 @@ def run_ours(args):
             "backward_and_fp8": dict(extra_paths, counting=(
                 "bwd: 2.5 x the kept-tile FLOPs of the forward (the five products dV, dP, S, dQ, dK per "
                 "kept pair against the forward's two; the kernels compute S and dP twice, which is not "
-                "counted); bf16 gradients; fp8: per-block e4m3 Q and K, bf16 P V")),
+                "counted); bf16 gradients; fp8: per-block e4m3 Q and K, bf16 P V; sparse_linear: the linear "
+                "branch and the alpha mix given the sparse output (features, per-head state, kept tiles and "
+                "totals), its TFLOP/s counted on the kept tiles' products alone")),
             "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         }

@@ -26,6 +26,7 @@ STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3:
 EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn_mask_noalloc",
             "sparse_attn_select", "sparse_attn_bwd_workspace_bytes", "sparse_attn_bwd",
             "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8",
+            "sparse_attn_sparse_linear_workspace_bytes", "sparse_attn_sparse_linear",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
             "sparse_attn_host", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_fwd_withheld_copy")
@@ -81,6 +82,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_quantize_fp8.restype = ctypes.c_int
         lib.sparse_attn_fwd_fp8.argtypes = [sp, vp, vp, f32p, f32p, vp, i32p, i32p, vp, ctypes.c_int, f32p, vp]
         lib.sparse_attn_fwd_fp8.restype = ctypes.c_int
+        lib.sparse_attn_sparse_linear_workspace_bytes.argtypes = [sp]
+        lib.sparse_attn_sparse_linear_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_sparse_linear.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, f32p, vp, ctypes.c_int, vp,
+                                                  ctypes.c_size_t, vp]
+        lib.sparse_attn_sparse_linear.restype = ctypes.c_int
         lib.sparse_attn_host_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
         lib.sparse_attn_host_workspace_bytes.restype = ctypes.c_size_t
         lib.sparse_attn_host.argtypes = [sp, vp, vp, vp, ctypes.c_double, ctypes.c_double, vp, ctypes.c_int,
@@ -365,6 +371,49 @@ def sparse_attn_fwd_fp8(q8: dict, V: torch.Tensor, cnt: torch.Tensor, idx: torch
                                             _ptr(lse), _stream(dev, stream))
     _check("sparse_attn_fwd_fp8", st)
     return (O, lse) if want_lse else O
+
+
+def sparse_linear_workspace_bytes(B, H, N, d, bq, bk) -> int:
+    shape = make_shape(B, H, N, d, bq, bk)
+    return int(load_library().sparse_attn_sparse_linear_workspace_bytes(ctypes.byref(shape)))
+
+
+def sparse_attn_sparse_linear(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, cnt: torch.Tensor,
+                              idx: torch.Tensor, O_s: torch.Tensor, alpha: torch.Tensor, bq: int, bk: int, *,
+                              out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """O = alpha * O_s + (1 - alpha) * O_l: O_s the sparse branch's output
+    (sparse_attn_fwd, bf16 or fp32; O takes its dtype), O_l linear attention
+    (elu + 1 features) over the complement of each row's kept blocks; alpha
+    fp32 [B, H, N]. d = 128."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = Q.device
+    for t, shp in ((cnt, (B, H, n_q)), (idx, (B, H, n_q, n_k))):
+        if t.dtype != torch.int32 or not t.is_contiguous() or tuple(t.shape) != shp or t.device != dev:
+            raise ValueError(f"index tensor must be contiguous int32 {shp} on {dev}")
+    if O_s.dtype not in (torch.bfloat16, torch.float32) or O_s.shape != Q.shape or not O_s.is_contiguous() \
+            or O_s.device != dev:
+        raise ValueError("O_s must be a contiguous bf16 or fp32 tensor of Q's shape")
+    if alpha.dtype != torch.float32 or tuple(alpha.shape) != (B, H, N) or not alpha.is_contiguous() \
+            or alpha.device != dev:
+        raise ValueError(f"alpha must be a contiguous fp32 tensor {(B, H, N)} on {dev}")
+    O = _out_tensor(Q, out, O_s.dtype)
+    lib = load_library()
+    shape = make_shape(B, H, N, d, bq, bk)
+    nbytes = int(lib.sparse_attn_sparse_linear_workspace_bytes(ctypes.byref(shape)))
+    if nbytes == 0:
+        raise ValueError("unsupported shape for the sparse + linear path (d must be 128)")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib.sparse_attn_sparse_linear(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), _ptr(cnt), _ptr(idx),
+                                       _ptr(O_s), _ptr(alpha), _ptr(O),
+                                       SA_F32 if O.dtype == torch.float32 else SA_BF16, _ptr(workspace), wbytes,
+                                       _stream(dev, stream))
+    _check("sparse_attn_sparse_linear", st)
+    return O
 
 
 def bwd_workspace_bytes(B, H, N, d, bq, bk) -> int:

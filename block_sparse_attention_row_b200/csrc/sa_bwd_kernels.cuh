@@ -71,19 +71,6 @@ enum WaitSite : unsigned int {
     W_LOADED = 0xD00B
 };
 
-__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int where, uint64_t lim) {
-    const bool w = mbar_wait_bounded(bar, parity, abort_flag, where, lim);
-    return __all_sync(0xFFFFFFFFu, w);
-}
-
-// Bounded wait for a copy already issued (abort path: it must land before the
-// CTA's shared memory is released).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t lim) {
-    for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < lim;) {
-    }
-}
-
 // ------------------------------------------------------------ prep kernels
 // Per query block (blockIdx.x = i, blockIdx.y = bh), one thread per row r:
 // lsed[(bh n_q + i) bq + r] = (LSE log2(e), D) with D = sum_c dO O, or
@@ -429,7 +416,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const Desc k_mn = desc_split(mnmajor_desc(smem_u32(smem + L::OFF_K), TILE_N * 128));
             // S is double-buffered: the products of tile g + 1 go out as soon as the
             // compute warps have read tile g's S and dP into registers.
-            const uint32_t tSb[2] = {tmem, tmem + 128};
+            // S buffer b at tmem + 128 b.
             const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
             int g = 0, kq = 0, rown = 0;
             bool ok = true;
@@ -451,7 +438,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     !mbar_wait_spin(&C.vch_full[cv], (gt / NVS) & 1, abort_flag, W_CH_FULL, lim))
                     return false;
                 tc_fence_after();
-                issue_sk(tSb[gt & 1], q_desc, k_desc, ck);
+                issue_sk(tmem + 128u * (gt & 1), q_desc, k_desc, ck);
                 issue_sk(tdP, do_desc, v_desc, cv);
                 umma_commit(&C.s_full);
                 umma_commit(&C.vch_empty[cv]);          // V is no longer needed
@@ -487,7 +474,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     const uint32_t coff = (uint32_t)(ck * L::TILE_BYTES) >> 4;
 #pragma unroll
                     for (int kk = 0; kk < TILE_N / 16; ++kk) bk[kk] = desc_at(k_mn, coff + ((kk * 16 * 128) >> 4));
-                    umma_ts_halves<TILE_N / 16>(tdQ, tSb[g & 1], tSb[g & 1] + 64, bk, IDESC_DQ, t > 0 ? 1u : 0u);
+                    const uint32_t tSg = tmem + 128u * (g & 1);
+                    umma_ts_halves<TILE_N / 16>(tdQ, tSg, tSg + 64, bk, IDESC_DQ, t > 0 ? 1u : 0u);
                     umma_commit(&C.ch_empty[ck]);          // K is no longer needed
                     if (t + 1 == nt) umma_commit(&C.o_full);
                     ++g;
@@ -505,7 +493,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int wq = warp & 3;                 // TMEM lane quarter
         const int row = wq * 32 + lane;          // query row within the tile
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t tSb[2] = {tmem + lane_off, tmem + 128 + lane_off};
+        // S buffer b at tmem + lane_off + 128 b.
         const uint32_t tdP = tmem + 256 + lane_off, tdQ = tmem + 384 + lane_off;
         const float sl2 = prm.scale_log2;
         const bool f32 = prm.out_f32 != 0;
@@ -540,7 +528,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 const int nvalid = j < 0 ? 0 : min(BK, prm.N - j * BK);
                 if (!wait_warp(&C.s_full, g & 1, abort_flag, W_S_FULL, lim)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t tS = tSb[g & 1];
+                const uint32_t tS = tmem + lane_off + 128u * (g & 1);
                 uint32_t s[64], dp[64];
                 tmem_ld64(tS + wg * 64, s);
                 tmem_ld64(tdP + wg * 64, dp);

@@ -19,6 +19,7 @@
 #include "sa_attn_kernel.cuh"
 #include "sa_bwd_kernels.cuh"
 #include "sa_fp8_kernels.cuh"
+#include "sa_linear_kernels.cuh"
 
 namespace {
 
@@ -419,9 +420,125 @@ sa_status launch_bwd(const Dims& g, const void* Q, const void* K, const void* V,
     return launch_bwd_t<64, 64>(g, Q, K, V, O, dO, lse, cnt, idx, dQ, dK, dV, out_f32, ws, st);
 }
 
+// ------------------------------------------------- sparse + linear (SLA2)
+struct LinWorkspace {
+    size_t pq, pk, zpart, hpart, hhi, hlo, z, total;
+    int n_b, splits, n_chunks;
+};
+
+LinWorkspace lin_layout(const Dims& g) {
+    LinWorkspace w;
+    w.n_b = (g.N + 63) / 64;
+    w.n_chunks = (g.N + sa::lin::LS_CHUNK - 1) / sa::lin::LS_CHUNK;
+    int sp = (sm_count() + g.BH - 1) / g.BH;   // about one wave of state CTAs
+    if (sp > w.n_chunks) sp = w.n_chunks;
+    w.splits = sp < 1 ? 1 : sp;
+    const size_t tok = (size_t)g.BH * g.N * g.d;
+    w.pq = 0;
+    w.pk = w.pq + round256(tok * 2);
+    w.zpart = w.pk + round256(tok * 2);
+    w.hpart = w.zpart + round256((size_t)g.BH * w.n_b * g.d * 4);
+    w.hhi = w.hpart + round256((size_t)g.BH * w.splits * g.d * g.d * 4);
+    w.hlo = w.hhi + round256((size_t)g.BH * g.d * g.d * 2);
+    w.z = w.hlo + round256((size_t)g.BH * g.d * g.d * 2);
+    w.total = w.z + round256((size_t)g.BH * g.d * 4);
+    return w;
+}
+
+template <int BQ>
+sa_status launch_sparse_linear(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
+                               const int32_t* idx, const void* Os, const float* alpha, void* O, bool out_f32,
+                               uint8_t* ws, cudaStream_t st) {
+    constexpr int D = 128;
+    const LinWorkspace w = lin_layout(g);
+    auto* pQ = reinterpret_cast<__nv_bfloat16*>(ws + w.pq);
+    auto* pK = reinterpret_cast<__nv_bfloat16*>(ws + w.pk);
+    float* zpart = reinterpret_cast<float*>(ws + w.zpart);
+    float* hpart = reinterpret_cast<float*>(ws + w.hpart);
+    auto* Hhi = reinterpret_cast<__nv_bfloat16*>(ws + w.hhi);
+    auto* Hlo = reinterpret_cast<__nv_bfloat16*>(ws + w.hlo);
+    float* z = reinterpret_cast<float*>(ws + w.z);
+    sa_status s;
+    sa::lin::phi_kernel<D><<<dim3(2 * w.n_b, g.BH), 128, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), pQ, pK, zpart, g.N, w.n_b);
+    if ((s = cuda_check(cudaGetLastError(), "phi_kernel launch")) != SA_OK) return s;
+
+    CUtensorMap m_pk128, m_v128;
+    if ((s = make_map(&m_pk128, pK, g, sa::lin::LS_CHUNK)) != SA_OK || (s = make_map(&m_v128, V, g, sa::lin::LS_CHUNK)) != SA_OK)
+        return s;
+    using LSL = sa::lin::LSLayout<D>;
+    auto kls = sa::lin::lin_state_kernel<D>;
+    if ((s = cuda_check(cudaFuncSetAttribute(kls, cudaFuncAttributeMaxDynamicSharedMemorySize, LSL::DYN_BYTES),
+                        "lin_state_kernel shared-memory attribute")) != SA_OK)
+        return s;
+    kls<<<dim3(g.BH, w.splits), sa::lin::LS_THREADS, LSL::DYN_BYTES, st>>>(m_pk128, m_v128, hpart, w.n_chunks, w.splits,
+                                                                          WAIT_LIMIT_NS);
+    if ((s = cuda_check(cudaGetLastError(), "lin_state_kernel launch")) != SA_OK) return s;
+    sa::lin::lin_finalize_kernel<D><<<g.BH, D, 0, st>>>(hpart, zpart, Hhi, Hlo, z, w.splits, w.n_b);
+    if ((s = cuda_check(cudaGetLastError(), "lin_finalize_kernel launch")) != SA_OK) return s;
+
+    CUtensorMap m_pq, m_pk, m_v, m_hhi, m_hlo;
+    Dims gh = g;
+    gh.N = D;   // H, viewed as D rows of D channels per head
+    if ((s = make_map(&m_pq, pQ, g, sa::lin::SL_MROWS)) != SA_OK || (s = make_map(&m_pk, pK, g, sa::lin::SL_BK)) != SA_OK ||
+        (s = make_map(&m_v, V, g, sa::lin::SL_BK)) != SA_OK || (s = make_map(&m_hhi, Hhi, gh, 128)) != SA_OK ||
+        (s = make_map(&m_hlo, Hlo, gh, 128)) != SA_OK)
+        return s;
+    using SLL = sa::lin::SLLayout<D>;
+    auto ksl = sa::lin::sparse_linear_kernel<D, BQ>;
+    if ((s = cuda_check(cudaFuncSetAttribute(ksl, cudaFuncAttributeMaxDynamicSharedMemorySize, SLL::DYN_BYTES),
+                        "sparse_linear_kernel shared-memory attribute")) != SA_OK)
+        return s;
+    sa::lin::SLParams prm;
+    prm.cnt = cnt;
+    prm.idx = idx;
+    prm.pQ = pQ;
+    prm.z = z;
+    prm.Os = Os;
+    prm.alpha = alpha;
+    prm.O = O;
+    prm.N = g.N;
+    prm.n_q = g.n_q;
+    prm.n_k = g.n_k;
+    prm.rows = g.BH * g.n_q;
+    prm.out_f32 = out_f32 ? 1 : 0;
+    prm.wait_limit_ns = WAIT_LIMIT_NS;
+    const int grid = prm.rows < sm_count() ? prm.rows : sm_count();
+    ksl<<<grid, sa::lin::SL_THREADS, SLL::DYN_BYTES, st>>>(m_pq, m_pk, m_v, m_hhi, m_hlo, prm);
+    return cuda_check(cudaGetLastError(), "sparse_linear_kernel launch");
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t sparse_attn_sparse_linear_workspace_bytes(const sa_shape* shape) {
+    Dims g;
+    if (check_shape(shape, g) != SA_OK || g.d != 128) return 0;
+    return lin_layout(g).total;
+}
+
+sa_status sparse_attn_sparse_linear(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                                    const int32_t* cnt, const int32_t* idx, const void* O_s, const float* alpha,
+                                    void* O, int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_fwd_args(shape, Q, K, V, cnt, idx, O, o_dtype, nullptr, g)) != SA_OK) return s;
+    if (g.d != 128) return fail(SA_ERR_UNSUPPORTED, "d=%d: the sparse + linear path supports d = 128", g.d);
+    if (!O_s || !alpha || !workspace) return fail(SA_ERR_INVALID_ARG, "NULL pointer among O_s, alpha, workspace");
+    if (!aligned16(O_s) || !aligned16(alpha) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required; 256 for workspace)");
+    const size_t need = lin_layout(g).total;
+    if (workspace_bytes < need)
+        return fail(SA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    const bool f32 = o_dtype == SA_F32;
+    s = (g.bq == 128) ? launch_sparse_linear<128>(g, Q, K, V, cnt, idx, O_s, alpha, O, f32, ws, st)
+                      : launch_sparse_linear<64>(g, Q, K, V, cnt, idx, O_s, alpha, O, f32, ws, st);
+    if (s != SA_OK) return s;
+    return ok();
+}
 
 size_t sparse_attn_bwd_workspace_bytes(const sa_shape* shape) {
     Dims g;

@@ -146,6 +146,20 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, v
     }
 }
 
+// mbar_wait_bounded by a whole warp; true only if every lane's wait succeeded.
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int where, uint64_t lim) {
+    const bool w = mbar_wait_bounded(bar, parity, abort_flag, where, lim);
+    return __all_sync(0xFFFFFFFFu, w);
+}
+
+// Bounded wait for a copy or product already issued (abort path: it must
+// land before the CTA's shared or tensor memory is released).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint64_t lim) {
+    for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < lim;) {
+    }
+}
+
 // --------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {

@@ -185,6 +185,41 @@ sa_status sparse_attn_fwd_fp8(const sa_shape* shape, const uint8_t* Q8, const ui
                               const int32_t* cnt, const int32_t* idx,
                               void* O, int o_dtype, float* lse_or_null, void* stream);
 
+/* Bytes of device workspace sparse_attn_sparse_linear needs for `shape`:
+ * phi(Q) and phi(K) in bf16 (2 * 2 * B*H*N*d), per-key-block sums of phi(k)
+ * (4 * B*H*ceil(N/64)*d), split partial states (4 * B*H*splits*d*d, splits
+ * about 148 / (B*H), at least 1), the state as a bf16 pair (2 * 2 * B*H*d*d)
+ * and z (4 * B*H*d), each rounded up to 256 bytes. 0 on an invalid shape or
+ * d != 128. */
+size_t sparse_attn_sparse_linear_workspace_bytes(const sa_shape* shape);
+
+/* The sparse + linear combination of "SLA2: Sparse-Linear Attention with
+ * Learnable Routing and QAT" §2A: O = alpha * O_s + (1 - alpha) * O_l, where
+ * O_s is the sparse branch (sparse_attn_fwd over the kept blocks, passed in)
+ * and O_l is linear attention over the complement of a row's kept blocks.
+ * The page prints no feature map; here phi(x) = elu(x) + 1 (positive), and
+ * for a query token t of query block i,
+ *   O_l(t) = sum_u (phi(q_t) . phi(k_u)) v_u / sum_u phi(q_t) . phi(k_u)
+ * over the valid key tokens u of the key blocks NOT in idx[i, 0:cnt[i]];
+ * O_l = 0 for a row that keeps every key block. It is computed as the total
+ * over all keys minus the kept part: the per-head state H = phi(K)^T V and
+ * z = sum_u phi(k_u) are built on the tensor cores (phi rounded to bf16, the
+ * operands of every product), and each row subtracts its kept tiles' sums
+ * inside the same fp32 accumulator. The result loses relative precision
+ * when the complement carries only a small part of the row's total linear
+ * weight (the subtraction cancels); on the workloads here it keeps at least
+ * 5% of it.
+ * Inputs:  Q, K, V bf16 [B,H,N,d] (d = 128, else SA_ERR_UNSUPPORTED); cnt,
+ *          idx as for sparse_attn_fwd; O_s [B,H,N,d] of type o_dtype (the
+ *          sparse branch's output); alpha fp32 [B,H,N], values in [0, 1].
+ * Output:  O [B,H,N,d] of type o_dtype.
+ * workspace: device, sparse_attn_sparse_linear_workspace_bytes(shape) bytes,
+ *          256-byte aligned; workspace_bytes is checked against that size. */
+sa_status sparse_attn_sparse_linear(const sa_shape* shape, const void* Q, const void* K,
+                                    const void* V, const int32_t* cnt, const int32_t* idx,
+                                    const void* O_s, const float* alpha, void* O, int o_dtype,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace sparse_attn_bwd needs for `shape`: the per-row
  * log-sum-exp and D = rowsum(dO * O) (8 * B*H * n_q * bq bytes), the
  * kept-block bitmap (4 * B*H * n_q * ceil(n_k/32)), and the transposed lists

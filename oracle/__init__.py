@@ -18,7 +18,9 @@ Sources (gist.science summaries; cited by page title and section):
   through, hence its backward pass in ``sparse_attn_backward``).
 * "SLA2: Sparse-Linear Attention with Learnable Routing and QAT": §1 Problem
   Statement and §2B Learnable Router (a compressed score computed from pooled
-  queries and keys).
+  queries and keys), §2A Faithful Sparse-Linear Formulation (the alpha mix of
+  a sparse and a linear branch: ``sparse_linear_oracle``) and §2C
+  Quantization-Aware Training (the low-bit sparse branch: ``sparse_attn_fp8``).
 * "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
   Semantic-Aware Permutation": §1 (mean or max pooling of contiguous token
   blocks) and §2B Centroid-Based Top-p Selection (sort by score, take items
@@ -47,11 +49,12 @@ from .sparse_attn_oracle import (
 from .sparse_attn_backward import attend_row_backward, block_sparse_attention_backward
 from .sparse_attn_fp8 import (block_sparse_attention_fp8, dequantize_blocks, e4m3_round,
                               quantize_blocks)
+from .sparse_linear_oracle import linear_row, phi, sparse_linear_attention
 
 __all__ = [
     "to_f64", "pool_blocks", "block_scores", "topk_count", "topp_threshold",
     "select_row", "hybrid_select", "hybrid_mask", "attend_row",
     "block_sparse_attention", "row_sample", "attend_row_backward",
     "block_sparse_attention_backward", "e4m3_round", "quantize_blocks", "dequantize_blocks",
-    "block_sparse_attention_fp8",
+    "block_sparse_attention_fp8", "phi", "linear_row", "sparse_linear_attention",
 ]

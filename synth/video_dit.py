@@ -171,3 +171,11 @@ def make_grad_out(B: int, H: int, N: int, d: int, *, seed: int, device="cpu") ->
     in fp32 from its own generator, rounded once to bf16, shape [B, H, N, d]."""
     gen = torch.Generator(device=device).manual_seed(seed)
     return torch.randn((B, H, N, d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def make_mix_ratio(B: int, H: int, N: int, *, seed: int, device="cpu") -> torch.Tensor:
+    """A seeded per-token mixing ratio alpha for the sparse + linear
+    combination (a stand-in for the learned vector): iid U[0, 1], fp32
+    [B, H, N], from its own generator."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    return torch.rand((B, H, N), generator=gen, device=device, dtype=torch.float32)

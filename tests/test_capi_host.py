@@ -201,3 +201,17 @@ def test_fp8_host_validation(lib):
     assert lib.sparse_attn_fwd_fp8(d128, a, a, a, a, a, a, a, a, 3, None, None) == 1   # o_dtype
     assert lib.sparse_attn_quantize_fp8(d128, a, a, a, z, a, a, None) == 1
     assert lib.sparse_attn_quantize_fp8(d128, a, a, a, ctypes.c_void_p(20), a, a, None) == 1
+
+
+def test_sparse_linear_host_validation(lib):
+    from block_sparse_attention_row_b200.capi import make_shape
+    a, z, ws = ctypes.c_void_p(16), ctypes.c_void_p(0), ctypes.c_void_p(256)
+    d128 = ctypes.byref(make_shape(1, 2, 4096, 128, 128, 64))
+    d64 = ctypes.byref(make_shape(1, 2, 4096, 64, 64, 64))
+    need = lib.sparse_attn_sparse_linear_workspace_bytes(d128)
+    assert need > 0 and lib.sparse_attn_sparse_linear_workspace_bytes(d64) == 0
+    assert lib.sparse_attn_sparse_linear(d64, a, a, a, a, a, a, a, a, 0, ws, need, None) == 2
+    assert lib.sparse_attn_sparse_linear(d128, a, a, a, a, a, z, a, a, 0, ws, need, None) == 1
+    assert lib.sparse_attn_sparse_linear(d128, a, a, a, a, a, a, a, a, 0, ws, need - 1, None) == 1
+    assert b"workspace" in lib.sparse_attn_last_error()
+    assert lib.sparse_attn_sparse_linear(d128, a, a, a, a, a, a, a, a, 0, ctypes.c_void_p(16), need, None) == 1

@@ -34,7 +34,10 @@
 //   dQ kernel:   S double-buffered [0,128) and [128,256), dP [256,384),
 //                dQ [384,384+d): the products of tile t+1 run while the compute
 //                warps turn tile t's S and dP (already in registers) into dS;
-//   dK/dV kernel: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512).
+//   dK/dV kernel: S^T in two 64-column buffers [0,128), dP^T likewise
+//                [128,256), dV [256,384), dK [384,512): a query block is taken in
+//                halves of 64 queries, the products of one half running while the
+//                compute warps form the previous half's P^T and dS^T.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -261,6 +264,7 @@ struct Ctrl {
     uint64_t s_full, p_full, o_full, acc_free, drain;
     uint64_t loaded;               // dQ kernel: the compute warps hold S and dP of a tile in registers
     uint64_t vch_full[2], vch_empty[2];   // dQ kernel: the V ring (the K ring uses ch_full/ch_empty)
+    uint64_t s2_full[2], p2_full[2];      // dK/dV kernel: per TMEM buffer of a 64-query unit
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -596,8 +600,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO, const Params prm) {
     using L = KVLayout<D, BQ>;
     constexpr int NST = L::NST;
-    constexpr int HALF = BQ / 2;             // query columns per warpgroup
-    constexpr int NCHUNK = HALF / 32;        // 32-column chunks per warpgroup
+    constexpr int NH = BQ / 64;              // 64-query units per query block
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Ctrl& C = *reinterpret_cast<Ctrl*>(smem + L::OFF_CTRL);
@@ -613,8 +616,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(&C.qs_full[s], 1);
             mbar_init(&C.qs_empty[s], 1);
         }
-        mbar_init(&C.s_full, 1);
-        mbar_init(&C.p_full, 8);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&C.s2_full[b], 1);
+            mbar_init(&C.p2_full[b], 8);
+        }
         mbar_init(&C.o_full, 1);
         mbar_init(&C.acc_free, 8);
         mbar_init(&C.drain, 1);
@@ -692,16 +697,20 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 for (int ee = (es > NST ? es - NST : 0); ee < es; ++ee) drain_wait(&C.qs_full[ee % NST], (ee / NST) & 1, lim);
             }
         } else if (warp == MMA_WARP && lane == 0) {
-            constexpr uint32_t IDESC_ST = make_idesc_bf16(MROWS, BQ, false);
+            // Query blocks are processed in halves of 64 queries ("units"); S^T
+            // and dP^T of a unit go to buffer unit & 1 (64 columns each), so the
+            // products of unit u+1 run while the compute warps form unit u's
+            // weights, and dV, dK of unit u follow.
+            constexpr uint32_t IDESC_ST = make_idesc_bf16(MROWS, 64, false);
             constexpr uint32_t IDESC_G = make_idesc_bf16(MROWS, D, true);
             const Desc k_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_K)));
             const Desc v_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_V)));
             const Desc st_desc = desc_split(kmajor_desc(smem_u32(smem + L::OFF_ST)));
             const Desc st_mn = desc_split(mnmajor_desc(smem_u32(smem + L::OFF_ST), BQ * 128));
-            const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
-            int itn = 0, es = 0, g = 0;
+            const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+            int itn = 0, es = 0, gu = 0;
             bool ok = true;
-            // d = A (K or V pair tile, 128 rows) times B^T (Q or dO of the stage).
+            // d = A (K or V pair tile, 128 rows) times B^T (64 rows of Q or dO at b_off16).
             auto issue_t = [&](uint32_t d, Desc a, uint32_t b_off16) {
 #pragma unroll
                 for (int sl = 0; sl < L::SLABS; ++sl)
@@ -711,38 +720,67 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                                 desc_at(st_desc, b_off16 + ((sl * (BQ * 128) + kk * 32) >> 4)), IDESC_ST,
                                 (sl | kk) ? 1u : 0u);
             };
+            // Offsets (16-byte units) of unit v's Q and dO rows in the stage ring.
+            auto q_off_of = [&](int e_glob, int hf) -> uint32_t {
+                return (uint32_t)((e_glob % NST) * 2 * L::QT_BYTES + hf * 64 * 128) >> 4;
+            };
+            // dV, dK of the unit gu_u (entry e_glob, half hf); first = it overwrites.
+            auto issue_grad = [&](int gu_u, int e_glob, int hf, bool first) {
+                const uint32_t qo = q_off_of(e_glob, hf);
+                const uint32_t doo = qo + ((uint32_t)L::QT_BYTES >> 4);
+                uint64_t bq_do[4], bq_q[4];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    bq_q[kk] = desc_at(st_mn, qo + ((kk * 16 * 128) >> 4));
+                    bq_do[kk] = desc_at(st_mn, doo + ((kk * 16 * 128) >> 4));
+                }
+                const uint32_t tSu = tmem + 64u * (gu_u & 1), tdPu = tmem + 128 + 64u * (gu_u & 1);
+                umma_ts_halves<4>(tdV, tSu, tSu + 32, bq_do, IDESC_G, first ? 0u : 1u);
+                umma_ts_halves<4>(tdK, tdPu, tdPu + 32, bq_q, IDESC_G, first ? 0u : 1u);
+                if (hf == NH - 1) umma_commit(&C.qs_empty[e_glob % NST]);
+            };
             for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
                 const int cnt = count_of(it);
                 if (cnt == 0) continue;
                 if (!mbar_wait_spin(&C.kv_full, itn & 1, abort_flag, W_KV_FULL, lim)) { ok = false; break; }
-                for (int e = 0; e < cnt; ++e) {
-                    const int st = es % NST;
-                    if (!mbar_wait_spin(&C.qs_full[st], (es / NST) & 1, abort_flag, W_Q_FULL, lim)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t q_off = (uint32_t)(st * 2 * L::QT_BYTES) >> 4;
-                    const uint32_t do_off = q_off + ((uint32_t)L::QT_BYTES >> 4);
-                    issue_t(tS, k_desc, q_off);
-                    issue_t(tdP, v_desc, do_off);
-                    umma_commit(&C.s_full);
-                    if (!mbar_wait_spin(&C.p_full, g & 1, abort_flag, W_P_FULL, lim)) { ok = false; break; }
-                    if (e == 0 && itn > 0 && !mbar_wait_spin(&C.acc_free, (itn - 1) & 1, abort_flag, W_ACC_FREE, lim)) {
+                const int nu = cnt * NH;
+                for (int v = 0; v < nu; ++v, ++gu) {
+                    const int e_glob = es + v / NH, hf = v % NH;
+                    if (hf == 0 &&
+                        !mbar_wait_spin(&C.qs_full[e_glob % NST], (e_glob / NST) & 1, abort_flag, W_Q_FULL, lim)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    uint64_t bq_do[BQ / 16], bq_q[BQ / 16];
-#pragma unroll
-                    for (int kk = 0; kk < BQ / 16; ++kk) {
-                        bq_q[kk] = desc_at(st_mn, q_off + ((kk * 16 * 128) >> 4));
-                        bq_do[kk] = desc_at(st_mn, do_off + ((kk * 16 * 128) >> 4));
+                    const uint32_t qo = q_off_of(e_glob, hf);
+                    issue_t(tmem + 64u * (gu & 1), k_desc, qo);
+                    issue_t(tmem + 128 + 64u * (gu & 1), v_desc, qo + ((uint32_t)L::QT_BYTES >> 4));
+                    umma_commit(&C.s2_full[gu & 1]);
+                    if (v >= 1) {
+                        const int pu = gu - 1, pe = es + (v - 1) / NH, ph = (v - 1) % NH;
+                        if (!mbar_wait_spin(&C.p2_full[pu & 1], (pu >> 1) & 1, abort_flag, W_P_FULL, lim) ||
+                            (v == 1 && itn > 0 &&
+                             !mbar_wait_spin(&C.acc_free, (itn - 1) & 1, abort_flag, W_ACC_FREE, lim))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_grad(pu, pe, ph, v == 1);
                     }
-                    umma_ts_halves<BQ / 16>(tdV, tS, tS + HALF, bq_do, IDESC_G, e > 0 ? 1u : 0u);
-                    umma_ts_halves<BQ / 16>(tdK, tdP, tdP + HALF, bq_q, IDESC_G, e > 0 ? 1u : 0u);
-                    umma_commit(&C.qs_empty[st]);
-                    ++es;
-                    ++g;
                 }
                 if (!ok) break;
+                // The item's last unit.
+                {
+                    const int pu = gu - 1, pe = es + (nu - 1) / NH, ph = (nu - 1) % NH;
+                    if (!mbar_wait_spin(&C.p2_full[pu & 1], (pu >> 1) & 1, abort_flag, W_P_FULL, lim) ||
+                        (nu == 1 && itn > 0 && !mbar_wait_spin(&C.acc_free, (itn - 1) & 1, abort_flag, W_ACC_FREE, lim))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_grad(pu, pe, ph, nu == 1);
+                }
+                es += cnt;
                 umma_commit(&C.o_full);
                 umma_commit(&C.kv_empty);
                 ++itn;
@@ -754,15 +792,14 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(COMPUTE_REGS));
-        const int wg = warp / 4;
+        const int wg = warp / 4;                 // 32 of a unit's 64 query columns each
         const int wq = warp & 3;
         const int row = wq * 32 + lane;          // key within the pair tile
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_off, tdP = tmem + 128 + lane_off;
         const uint32_t tdV = tmem + 256 + lane_off, tdK = tmem + 384 + lane_off;
         const float sl2 = prm.scale_log2;
         const bool f32 = prm.out_f32 != 0;
-        int itn = 0, es = 0, g = 0;
+        int itn = 0, es = 0, gu = 0;
         bool ok = true;
         for (int it = blockIdx.x; ok && it < items; it += gridDim.x) {
             const int cnt = count_of(it);
@@ -781,41 +818,38 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if ((e & 31) == 0) window = entry_of(it, cnt, e + lane);
                 const int ent = __shfl_sync(0xFFFFFFFFu, window, e & 31);
                 const bool kept = key_valid && ((ent >> half) & 1);
-                const int st = es % NST;
+                const int eg = es + e, st = eg % NST;
                 // The stage's LSE and D values are read from shared memory: wait for its copy too.
-                if (!wait_warp(&C.qs_full[st], (es / NST) & 1, abort_flag, W_Q_FULL, lim) ||
-                    !wait_warp(&C.s_full, g & 1, abort_flag, W_S_FULL, lim)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+                if (!wait_warp(&C.qs_full[st], (eg / NST) & 1, abort_flag, W_Q_FULL, lim)) { ok = false; break; }
                 const float2* lsed = reinterpret_cast<const float2*>(smem + L::OFF_LSED + st * L::LSED_BYTES);
-#pragma unroll
-                for (int h = 0; h < NCHUNK; ++h) {
-                    const int col = wg * HALF + h * 32;   // query columns [col, col + 32)
+                for (int hf = 0; hf < NH; ++hf, ++gu) {
+                    const int b = gu & 1;
+                    if (!wait_warp(&C.s2_full[b], (gu >> 1) & 1, abort_flag, W_S_FULL, lim)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t tS = tmem + lane_off + 64u * b, tdP = tmem + 128 + lane_off + 64u * b;
                     uint32_t s[32], dp[32];
-                    tmem_ld32(tS + col, s);
-                    tmem_ld32(tdP + col, dp);
+                    tmem_ld32(tS + wg * 32, s);
+                    tmem_ld32(tdP + wg * 32, dp);
                     float l2[32], dv[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const float2 v = lsed[col + c];
+                        const float2 v = lsed[hf * 64 + wg * 32 + c];
                         l2[c] = v.x;
                         dv[c] = v.y;
                     }
                     uint32_t pk[16], dk[16];
                     p_ds_chunk(s, dp, l2, dv, kept ? 0xFFFFFFFFu : 0u, sl2, pk, dk);
                     // Over this warpgroup's own S^T and dP^T columns (already read).
-                    tmem_st16_nowait(tS + wg * HALF + h * 16, pk);
-                    tmem_st16_nowait(tdP + wg * HALF + h * 16, dk);
+                    tmem_st16_nowait(tS + wg * 32, pk);
+                    tmem_st16_nowait(tdP + wg * 32, dk);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&C.p2_full[b]);
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&C.p_full);
-                ++es;
-                ++g;
+                if (!ok) break;
             }
+            es += cnt;
             if (!ok) break;
             if (!wait_warp(&C.o_full, itn & 1, abort_flag, W_O_FULL, lim)) { ok = false; break; }
             tc_fence_after();

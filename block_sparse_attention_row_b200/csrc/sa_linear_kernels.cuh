@@ -254,7 +254,7 @@ namespace lin {
 //   l     = sum over kept tiles of rowsum(phi(Q_i) phi(K_t)^T)
 //   O_l   = O_acc / (phi(q) . z - l), or 0 when every key block is kept
 //   O     = alpha * O_s + (1 - alpha) * O_l
-// One row pipeline per CTA, rows assigned in contiguous runs. 192 threads:
+// One row pipeline per CTA, rows interleaved over the CTAs. 192 threads:
 // warps 0-3 the elementwise step and epilogue (one query row per thread,
 // one TMEM lane), warp 4 the TMA producer, warp 5 the tcgen05 issuer.
 // TMEM: S double-buffered [0, 128) and [128, 256) (the kept tile's
@@ -336,9 +336,9 @@ sparse_linear_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_cons
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int n_k = prm.n_k;
     const uint64_t lim = prm.wait_limit_ns;
-    // Contiguous runs of rows: consecutive rows of a CTA share a head.
-    const int per = (prm.rows + gridDim.x - 1) / gridDim.x;
-    const int r_begin = blockIdx.x * per, r_end = min(prm.rows, r_begin + per);
+    // Rows interleaved over the CTAs (r = blockIdx.x + k gridDim.x): at any time
+    // the grid works on one or two heads, whose phi(K) and V stay in L2.
+    const int r_begin = blockIdx.x, r_end = prm.rows, r_step = gridDim.x;
 
     if (threadIdx.x == 0) {
         mbar_init(&C.q_full, 1);
@@ -373,7 +373,7 @@ sparse_linear_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_cons
         // -------------------------------------------------------- producer
         int g = 0, kq = 0, gk = 0, gv = 0;
         bool ok = true;
-        for (int r = r_begin; ok && r < r_end; ++r) {
+        for (int r = r_begin; ok && r < r_end; r += r_step) {
             const int cnt = sl_count(prm, r);
             const int nt = (cnt + 1) / 2;
             const int bh = r / prm.n_q, qb = r % prm.n_q;
@@ -460,7 +460,7 @@ sparse_linear_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_cons
                 umma_commit(&C.k_empty[sk]);
                 return true;
             };
-            for (int r = r_begin; ok && r < r_end; ++r) {
+            for (int r = r_begin; ok && r < r_end; r += r_step) {
                 const int nt = (sl_count(prm, r) + 1) / 2;
                 if (!mbar_wait_spin(&C.q_full, kq & 1, abort_flag, SL_W_Q, lim)) { ok = false; break; }
                 ++kq;
@@ -522,7 +522,7 @@ sparse_linear_kernel(const __grid_constant__ CUtensorMap tmPQ, const __grid_cons
         const bool f32 = prm.out_f32 != 0;
         int g = 0, rown = 0;
         bool ok = true;
-        for (int r = r_begin; ok && r < r_end; ++r) {
+        for (int r = r_begin; ok && r < r_end; r += r_step) {
             const int cnt = sl_count(prm, r);
             const int nt = (cnt + 1) / 2;
             const int bh = r / prm.n_q, qb = r % prm.n_q;

@@ -23,7 +23,8 @@ Sources (gist.science summaries; cited by page title and section):
   Quantization-Aware Training (the low-bit sparse branch: ``sparse_attn_fp8``).
 * "Sparse VideoGen2: Accelerate Video Generation with Sparse Attention via
   Semantic-Aware Permutation": §1 (mean or max pooling of contiguous token
-  blocks) and §2B Centroid-Based Top-p Selection (sort by score, take items
+  blocks), §2A Semantic-Aware Permutation (k-means clustering and reordering of
+  the tokens: ``svg_permutation_oracle``) and §2B Centroid-Based Top-p Selection (sort by score, take items
   until the cumulative score reaches p).
 
 Parity pins: every forward function here is pinned by
@@ -50,6 +51,7 @@ from .sparse_attn_backward import attend_row_backward, block_sparse_attention_ba
 from .sparse_attn_fp8 import (block_sparse_attention_fp8, dequantize_blocks, e4m3_round,
                               quantize_blocks)
 from .sparse_linear_oracle import linear_row, phi, sparse_linear_attention
+from .svg_permutation_oracle import kmeans_permutation, permuted_sparse_attention
 
 __all__ = [
     "to_f64", "pool_blocks", "block_scores", "topk_count", "topp_threshold",
@@ -57,4 +59,5 @@ __all__ = [
     "block_sparse_attention", "row_sample", "attend_row_backward",
     "block_sparse_attention_backward", "e4m3_round", "quantize_blocks", "dequantize_blocks",
     "block_sparse_attention_fp8", "phi", "linear_row", "sparse_linear_attention",
+    "kmeans_permutation", "permuted_sparse_attention",
 ]

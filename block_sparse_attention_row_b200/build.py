@@ -13,7 +13,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libsparse_attn.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["sa_lib.cu"]
-DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_attn_kernel.cuh", "sa_bwd_kernels.cuh", "sa_fp8_kernels.cuh", "sa_linear_kernels.cuh",
+DEPS = ["sa_lib.cu", "sa_ptx.cuh", "sa_mask_kernels.cuh", "sa_attn_kernel.cuh", "sa_bwd_kernels.cuh", "sa_fp8_kernels.cuh", "sa_linear_kernels.cuh", "sa_kmeans_kernels.cuh",
         "sa_status_codes.h"]
 
 

@@ -27,6 +27,7 @@ EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn
             "sparse_attn_select", "sparse_attn_bwd_workspace_bytes", "sparse_attn_bwd",
             "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8",
             "sparse_attn_sparse_linear_workspace_bytes", "sparse_attn_sparse_linear",
+            "sparse_attn_kmeans_workspace_bytes", "sparse_attn_kmeans_permutation", "sparse_attn_permute_rows",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
             "sparse_attn_host", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_fwd_withheld_copy")
@@ -87,6 +88,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_sparse_linear.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, f32p, vp, ctypes.c_int, vp,
                                                   ctypes.c_size_t, vp]
         lib.sparse_attn_sparse_linear.restype = ctypes.c_int
+        lib.sparse_attn_kmeans_workspace_bytes.argtypes = [sp, ctypes.c_int]
+        lib.sparse_attn_kmeans_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_kmeans_permutation.argtypes = [sp, vp, ctypes.c_int, ctypes.c_int, f32p, i32p, i32p, f32p,
+                                                       vp, ctypes.c_size_t, vp]
+        lib.sparse_attn_kmeans_permutation.restype = ctypes.c_int
+        lib.sparse_attn_permute_rows.argtypes = [sp, vp, i32p, vp, ctypes.c_int, ctypes.c_int, vp]
+        lib.sparse_attn_permute_rows.restype = ctypes.c_int
         lib.sparse_attn_host_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
         lib.sparse_attn_host_workspace_bytes.restype = ctypes.c_size_t
         lib.sparse_attn_host.argtypes = [sp, vp, vp, vp, ctypes.c_double, ctypes.c_double, vp, ctypes.c_int,
@@ -416,6 +424,65 @@ def sparse_attn_sparse_linear(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     return O
 
 
+def kmeans_workspace_bytes(B, H, N, d, C, bq: int = 64, bk: int = 64) -> int:
+    shape = make_shape(B, H, N, d, bq, bk)
+    return int(load_library().sparse_attn_kmeans_workspace_bytes(ctypes.byref(shape), int(C)))
+
+
+def sparse_attn_kmeans_permutation(X: torch.Tensor, C: int, iters: int, *, init: Optional[torch.Tensor] = None,
+                                   workspace: Optional[torch.Tensor] = None, stream=None):
+    """k-means of every head's token vectors (Sparse VideoGen2 §2A) and the
+    stable permutation by cluster. X bf16 [B, H, N, d]; init fp32
+    [B, H, C, d] (cached centroids) or None. Returns (ids int32 [B, H, N],
+    perm int32 [B, H, N], centroids fp32 [B, H, C, d])."""
+    if not isinstance(X, torch.Tensor) or not X.is_cuda or X.dtype != torch.bfloat16 or X.dim() != 4 \
+            or not X.is_contiguous():
+        raise ValueError("X must be a contiguous bf16 CUDA tensor [B, H, N, d]")
+    B, H, N, d = X.shape
+    dev = X.device
+    if init is not None and (init.dtype != torch.float32 or tuple(init.shape) != (B, H, int(C), d)
+                             or not init.is_contiguous() or init.device != dev):
+        raise ValueError(f"init must be a contiguous fp32 tensor {(B, H, int(C), d)} on {dev}")
+    lib = load_library()
+    shape = make_shape(B, H, N, d, 64, 64)
+    nbytes = int(lib.sparse_attn_kmeans_workspace_bytes(ctypes.byref(shape), int(C)))
+    if nbytes == 0:
+        raise ValueError(f"unsupported shape or C={C} for the k-means permutation")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    ids = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    perm = torch.empty((B, H, N), dtype=torch.int32, device=dev)
+    M = torch.empty((B, H, int(C), d), dtype=torch.float32, device=dev)
+    st = lib.sparse_attn_kmeans_permutation(ctypes.byref(shape), _ptr(X), int(C), int(iters), _ptr(init),
+                                            _ptr(ids), _ptr(perm), _ptr(M), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(), _stream(dev, stream))
+    _check("sparse_attn_kmeans_permutation", st)
+    return ids, perm, M
+
+
+def sparse_attn_permute_rows(X: torch.Tensor, perm: torch.Tensor, *, inverse: bool = False,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y[b, h, i] = X[b, h, perm[b, h, i]] (inverse: Y[b, h, perm[b, h, i]] =
+    X[b, h, i]). X bf16 or fp32 [B, H, N, d]; perm int32 [B, H, N]."""
+    if not isinstance(X, torch.Tensor) or not X.is_cuda or X.dtype not in (torch.bfloat16, torch.float32) \
+            or X.dim() != 4 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous bf16 or fp32 CUDA tensor [B, H, N, d]")
+    B, H, N, d = X.shape
+    dev = X.device
+    if perm.dtype != torch.int32 or tuple(perm.shape) != (B, H, N) or not perm.is_contiguous() \
+            or perm.device != dev:
+        raise ValueError(f"perm must be a contiguous int32 tensor {(B, H, N)} on {dev}")
+    Y = _out_tensor(X, out, X.dtype)
+    if Y.data_ptr() == X.data_ptr():
+        raise ValueError("out must not be X")
+    shape = make_shape(B, H, N, d, 64, 64)
+    st = load_library().sparse_attn_permute_rows(ctypes.byref(shape), _ptr(X), _ptr(perm), _ptr(Y),
+                                                 SA_F32 if X.dtype == torch.float32 else SA_BF16,
+                                                 1 if inverse else 0, _stream(dev, stream))
+    _check("sparse_attn_permute_rows", st)
+    return Y
+
+
 def bwd_workspace_bytes(B, H, N, d, bq, bk) -> int:
     shape = make_shape(B, H, N, d, bq, bk)
     return int(load_library().sparse_attn_bwd_workspace_bytes(ctypes.byref(shape)))
@@ -465,6 +532,26 @@ def sparse_attn(Q, K, V, bq: int, bk: int, k: float, p: float, *, stream=None):
     m = sparse_attn_mask(Q, K, bq, bk, k, p, stream=stream)
     O = sparse_attn_fwd(Q, K, V, m["cnt"], m["idx"], bq, bk, stream=stream)
     return O, m["cnt"], m["idx"]
+
+
+def permuted_sparse_attn(Q, K, V, bq: int, bk: int, k: float, p: float, C_q: int, C_k: int, iters: int, *,
+                         init_q: Optional[torch.Tensor] = None, init_k: Optional[torch.Tensor] = None,
+                         stream=None) -> dict:
+    """Sparse VideoGen2 §2A ahead of the path: Q and K clustered independently
+    (k-means, C_q and C_k clusters, `iters` rounds, optional cached centroids),
+    Q rows and K, V rows gathered into cluster order, the mask and block-sparse
+    forward run on the permuted sequences, and O scattered back to token order.
+    Returns {"O", "cnt", "idx" (of the permuted sequence), "perm_q", "perm_k",
+    "centroids_q", "centroids_k"}."""
+    _, perm_q, Mq = sparse_attn_kmeans_permutation(Q, C_q, iters, init=init_q, stream=stream)
+    _, perm_k, Mk = sparse_attn_kmeans_permutation(K, C_k, iters, init=init_k, stream=stream)
+    Qp = sparse_attn_permute_rows(Q, perm_q, stream=stream)
+    Kp = sparse_attn_permute_rows(K, perm_k, stream=stream)
+    Vp = sparse_attn_permute_rows(V, perm_k, stream=stream)
+    Op, cnt, idx = sparse_attn(Qp, Kp, Vp, bq, bk, k, p, stream=stream)
+    O = sparse_attn_permute_rows(Op, perm_q, inverse=True, stream=stream)
+    return {"O": O, "cnt": cnt, "idx": idx, "perm_q": perm_q, "perm_k": perm_k,
+            "centroids_q": Mq, "centroids_k": Mk}
 
 
 def host_workspace_bytes(B: int, H: int, N: int, d: int, bq: int, bk: int,

@@ -20,6 +20,7 @@
 #include "sa_bwd_kernels.cuh"
 #include "sa_fp8_kernels.cuh"
 #include "sa_linear_kernels.cuh"
+#include "sa_kmeans_kernels.cuh"
 
 namespace {
 
@@ -508,9 +509,97 @@ sa_status launch_sparse_linear(const Dims& g, const void* Q, const void* K, cons
     return cuda_check(cudaGetLastError(), "sparse_linear_kernel launch");
 }
 
+// ------------------------------------------- semantic-aware permutation
+constexpr int KM_MAX_C = 8192;
+constexpr int KM_MAX_ITERS = 100;
+
+sa_status check_kmeans(const sa_shape* shape, int C, int iters, Dims& g) {
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if (C < 1 || C > g.N || C > KM_MAX_C)
+        return fail(SA_ERR_INVALID_ARG, "C=%d clusters: need 1 <= C <= min(N=%d, %d)", C, g.N, KM_MAX_C);
+    if (iters < 0 || iters > KM_MAX_ITERS) return fail(SA_ERR_INVALID_ARG, "iters=%d outside [0, %d]", iters, KM_MAX_ITERS);
+    return SA_OK;
+}
+
+template <int D>
+sa_status launch_kmeans(const Dims& g, const void* X, int C, int iters, const float* init, int32_t* ids,
+                        int32_t* perm, float* M, int32_t* off, cudaStream_t st) {
+    auto* x = reinterpret_cast<const __nv_bfloat16*>(X);
+    sa_status s;
+    if (init) {
+        if ((s = cuda_check(cudaMemcpyAsync(M, init, (size_t)g.BH * C * D * sizeof(float), cudaMemcpyDeviceToDevice, st),
+                            "copy the initial centroids")) != SA_OK)
+            return s;
+    } else {
+        sa::km::km_init_kernel<D><<<dim3(C, g.BH), D, 0, st>>>(x, M, g.N, C);
+        if ((s = cuda_check(cudaGetLastError(), "km_init_kernel launch")) != SA_OK) return s;
+    }
+    const dim3 ag((g.N + sa::km::AS_THREADS - 1) / sa::km::AS_THREADS, g.BH);
+    for (int it = 0; it <= iters; ++it) {
+        sa::km::km_assign_kernel<D><<<ag, sa::km::AS_THREADS, 0, st>>>(x, M, ids, g.N, C);
+        if ((s = cuda_check(cudaGetLastError(), "km_assign_kernel launch")) != SA_OK) return s;
+        sa::km::km_sort_kernel<<<g.BH, 32, (size_t)C * sizeof(int32_t), st>>>(ids, perm, off, g.N, C);
+        if ((s = cuda_check(cudaGetLastError(), "km_sort_kernel launch")) != SA_OK) return s;
+        if (it == iters) break;   // the final assignment is not followed by an update
+        sa::km::km_update_kernel<D><<<dim3(C, g.BH), D, 0, st>>>(x, perm, off, M, g.N, C);
+        if ((s = cuda_check(cudaGetLastError(), "km_update_kernel launch")) != SA_OK) return s;
+    }
+    return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t sparse_attn_kmeans_workspace_bytes(const sa_shape* shape, int C) {
+    Dims g;
+    if (check_kmeans(shape, C, 0, g) != SA_OK) return 0;
+    return round256((size_t)g.BH * (C + 1) * sizeof(int32_t));
+}
+
+sa_status sparse_attn_kmeans_permutation(const sa_shape* shape, const void* X, int C, int iters,
+                                         const float* init_or_null, int32_t* ids, int32_t* perm, float* centroids,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_kmeans(shape, C, iters, g)) != SA_OK) return s;
+    if (!X || !ids || !perm || !centroids || !workspace)
+        return fail(SA_ERR_INVALID_ARG, "NULL pointer among X, ids, perm, centroids, workspace");
+    if (!aligned16(X) || !aligned16(ids) || !aligned16(perm) || !aligned16(centroids) ||
+        (init_or_null && !aligned16(init_or_null)) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required; 256 for workspace)");
+    const size_t need = round256((size_t)g.BH * (C + 1) * sizeof(int32_t));
+    if (workspace_bytes < need) return fail(SA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, need);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* off = reinterpret_cast<int32_t*>(workspace);
+    s = (g.d == 128) ? launch_kmeans<128>(g, X, C, iters, init_or_null, ids, perm, centroids, off, st)
+                     : launch_kmeans<64>(g, X, C, iters, init_or_null, ids, perm, centroids, off, st);
+    if (s != SA_OK) return s;
+    return ok();
+}
+
+sa_status sparse_attn_permute_rows(const sa_shape* shape, const void* X, const int32_t* perm, void* Y, int dtype,
+                                   int inverse, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_shape(shape, g)) != SA_OK) return s;
+    if ((s = check_out_dtype(dtype)) != SA_OK) return s;
+    if (!X || !perm || !Y) return fail(SA_ERR_INVALID_ARG, "NULL pointer among X, perm, Y");
+    if (X == Y) return fail(SA_ERR_INVALID_ARG, "X and Y must not be the same buffer");
+    if (!aligned16(X) || !aligned16(perm) || !aligned16(Y))
+        return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const dim3 grid((g.N + 7) / 8, g.BH);
+    auto* x = reinterpret_cast<const uint8_t*>(X);
+    auto* y = reinterpret_cast<uint8_t*>(Y);
+    const int row_bytes = g.d * (dtype == SA_F32 ? 4 : 2);
+    if (row_bytes == 128) sa::km::permute_rows_kernel<128><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
+    else if (row_bytes == 256) sa::km::permute_rows_kernel<256><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
+    else sa::km::permute_rows_kernel<512><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
+    if ((s = cuda_check(cudaGetLastError(), "permute_rows_kernel launch")) != SA_OK) return s;
+    return ok();
+}
 
 size_t sparse_attn_sparse_linear_workspace_bytes(const sa_shape* shape) {
     Dims g;

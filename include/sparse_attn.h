@@ -185,6 +185,58 @@ sa_status sparse_attn_fwd_fp8(const sa_shape* shape, const uint8_t* Q8, const ui
                               const int32_t* cnt, const int32_t* idx,
                               void* O, int o_dtype, float* lse_or_null, void* stream);
 
+/* Bytes of device workspace sparse_attn_kmeans_permutation needs: the
+ * cluster offsets, 4 * B*H*(C + 1) rounded up to 256. 0 on an invalid shape
+ * or C. */
+size_t sparse_attn_kmeans_workspace_bytes(const sa_shape* shape, int C);
+
+/* Semantic-aware permutation of "Sparse VideoGen2: Accelerate Video
+ * Generation with Sparse Attention via Semantic-Aware Permutation" §2A: the
+ * N token vectors of every (b, h) are clustered by k-means into C clusters
+ * and listed cluster by cluster, so that a block of the permuted sequence
+ * holds tokens of one cluster (Q and K are permuted independently; V takes
+ * K's permutation). §2C starts k-means from the previous step's centroids:
+ * init_or_null. The page fixes no initialisation, distance or tie rule; here
+ * (so that the result is exact and reproducible):
+ *   start     centroid c = the token at floor(c N / C), unless init is given;
+ *   assign    squared Euclidean distance summed over the channels in order,
+ *             each subtraction, product and addition rounded to fp32 (no
+ *             fused multiply-add); the nearest centroid, ties to the lower
+ *             index;
+ *   update    the fp32 sum of a cluster's members in ascending token order,
+ *             divided by their count; an empty cluster keeps its centroid;
+ *   iters     `iters` rounds of (assign, update), then a final assign;
+ *   perm      tokens sorted by final cluster id, ascending token order within
+ *             a cluster (a stable sort): perm[i] is the token at position i.
+ * Inputs:  shape (B, H, N, d with d in {64, 128}; bq and bk are checked as
+ *          elsewhere but unused); X bf16 [B,H,N,d]; C clusters, 1 <= C <=
+ *          min(N, 8192); iters in [0, 100]; init_or_null fp32 [B,H,C,d].
+ * Outputs: ids int32 [B,H,N] (final cluster of every token), perm int32
+ *          [B,H,N], centroids fp32 [B,H,C,d] (after `iters` updates; may be
+ *          the same buffer as init_or_null).
+ * workspace: device, sparse_attn_kmeans_workspace_bytes(shape, C) bytes,
+ *          256-byte aligned; workspace_bytes is checked against that size.
+ * Device pointers 16-byte aligned. Errors: SA_ERR_INVALID_ARG on a bad
+ * shape, C, iters, pointer or workspace; SA_ERR_CUDA on a failed launch. */
+sa_status sparse_attn_kmeans_permutation(const sa_shape* shape, const void* X, int C, int iters,
+                                         const float* init_or_null, int32_t* ids, int32_t* perm,
+                                         float* centroids, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/* Row permutation of [B,H,N,d] for the semantic-aware permutation (Sparse
+ * VideoGen2 §2A): inverse = 0 gathers Y[b,h,i] = X[b,h,perm[b,h,i]] (tokens
+ * into cluster order), inverse = 1 scatters Y[b,h,perm[b,h,i]] = X[b,h,i]
+ * (an output in cluster order back to token order). Rows are copied bit for
+ * bit. dtype: SA_BF16 or SA_F32, the element type of X and Y. perm must be a
+ * permutation of 0..N-1 for every (b, h) (the result of
+ * sparse_attn_kmeans_permutation); an entry outside [0, N) is skipped and
+ * reported as SA_ERR_DEVICE_ASSERT by sparse_attn_check_device_error (a
+ * repeated entry leaves some rows of Y unwritten and is not detected).
+ * X and Y distinct, device pointers 16-byte aligned.
+ * Errors: SA_ERR_INVALID_ARG on a bad shape, dtype or pointer. */
+sa_status sparse_attn_permute_rows(const sa_shape* shape, const void* X, const int32_t* perm,
+                                   void* Y, int dtype, int inverse, void* stream);
+
 /* Bytes of device workspace sparse_attn_sparse_linear needs for `shape`:
  * phi(Q) and phi(K) in bf16 (2 * 2 * B*H*N*d), per-key-block sums of phi(k)
  * (4 * B*H*ceil(N/64)*d), split partial states (4 * B*H*splits*d*d, splits

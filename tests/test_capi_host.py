@@ -215,3 +215,37 @@ def test_sparse_linear_host_validation(lib):
     assert lib.sparse_attn_sparse_linear(d128, a, a, a, a, a, a, a, a, 0, ws, need - 1, None) == 1
     assert b"workspace" in lib.sparse_attn_last_error()
     assert lib.sparse_attn_sparse_linear(d128, a, a, a, a, a, a, a, a, 0, ctypes.c_void_p(16), need, None) == 1
+
+
+def test_kmeans_host_validation(lib):
+    from block_sparse_attention_row_b200.capi import make_shape
+    a, z, ws = ctypes.c_void_p(16), ctypes.c_void_p(0), ctypes.c_void_p(256)
+    sh = ctypes.byref(make_shape(1, 2, 1000, 128, 64, 64))
+    need = lib.sparse_attn_kmeans_workspace_bytes(sh, 100)
+    assert need == ((2 * 101 * 4 + 255) // 256) * 256
+    for C in (0, -1, 1001):
+        assert lib.sparse_attn_kmeans_workspace_bytes(sh, C) == 0
+    assert lib.sparse_attn_kmeans_workspace_bytes(ctypes.byref(make_shape(1, 2, 1000, 96, 64, 64)), 10) == 0
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 1001, 5, None, a, a, a, ws, need, None) == 1
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 100, 101, None, a, a, a, ws, need, None) == 1
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 100, -1, None, a, a, a, ws, need, None) == 1
+    assert lib.sparse_attn_kmeans_permutation(sh, z, 100, 5, None, a, a, a, ws, need, None) == 1
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 100, 5, None, a, a, a, ws, need - 1, None) == 1
+    assert b"workspace" in lib.sparse_attn_last_error()
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 100, 5, None, a, a, a, ctypes.c_void_p(16), need, None) == 1
+    assert lib.sparse_attn_kmeans_permutation(sh, a, 100, 5, ctypes.c_void_p(8), a, a, a, ws, need, None) == 1
+    # Row permutation: dtype, aliasing, null and alignment are refused before any launch.
+    assert lib.sparse_attn_permute_rows(sh, a, a, ctypes.c_void_p(32), 2, 0, None) == 1
+    assert lib.sparse_attn_permute_rows(sh, a, a, a, 0, 0, None) == 1
+    assert lib.sparse_attn_permute_rows(sh, a, z, ctypes.c_void_p(32), 0, 0, None) == 1
+    assert lib.sparse_attn_permute_rows(sh, a, a, ctypes.c_void_p(40), 0, 0, None) == 1
+
+
+def test_kmeans_binding_refuses_cpu_tensors():
+    import torch
+    from block_sparse_attention_row_b200 import sparse_attn_kmeans_permutation, sparse_attn_permute_rows
+    X = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sparse_attn_kmeans_permutation(X, 4, 2)
+    with pytest.raises(ValueError):
+        sparse_attn_permute_rows(X, torch.zeros(1, 1, 64, dtype=torch.int32))

@@ -31,6 +31,12 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse attn ms/call & kept-tile TFLOPS vs bf16 peak; speedup vs own dense"
 UNIT = "TFLOP/s (kept tiles)"
 DEFAULT_CONFIG = "wan"
+# Semantic-aware permutation timed beside the path: clusters per head for Q
+# and for K, k-means rounds from token positions (cold) and from cached
+# centroids (warm).
+PERM_C = 256
+PERM_COLD_ITERS = 8
+PERM_WARM_ITERS = 2
 FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_attn_kernel.cuh",
                "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
 MASK_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
@@ -517,6 +523,71 @@ def run_ours(args):
                               "sparse_linear_kept_tile_tflops": fl_t / (sl_ms * 1e-3) / 1e12})
             extra_paths[tag] = entry
         check_device_error(dev)
+        # Semantic-aware permutation (Sparse VideoGen2 §2A, §2C) ahead of the
+        # same mask and forward at the workload's (k, p): k-means of Q and of K
+        # (PERM_C clusters each), cold (centroids at token positions, 8 rounds)
+        # and warm (from the cold run's centroids, as the centroid cache does,
+        # 2 rounds); the Q, K, V gathers, the mask and forward on the permuted
+        # sequences and the scatter of O back to token order.
+        from block_sparse_attention_row_b200 import (kmeans_workspace_bytes, sparse_attn_kmeans_permutation,
+                                                     sparse_attn_permute_rows)
+        kws = torch.empty(kmeans_workspace_bytes(B, H, N, d, PERM_C), dtype=torch.uint8, device=dev)
+        _, pq, Mq = sparse_attn_kmeans_permutation(Q, PERM_C, PERM_COLD_ITERS, workspace=kws)
+        _, pk, Mk = sparse_attn_kmeans_permutation(K, PERM_C, PERM_COLD_ITERS, workspace=kws)
+        Qp, Kp, Vp, Op = (torch.empty_like(Q) for _ in range(4))
+        outp = {"cnt": torch.empty_like(out["cnt"]), "idx": torch.empty_like(out["idx"])}
+        O_tok = torch.empty_like(O)
+
+        def do_km_cold():
+            sparse_attn_kmeans_permutation(Q, PERM_C, PERM_COLD_ITERS, workspace=kws)
+            sparse_attn_kmeans_permutation(K, PERM_C, PERM_COLD_ITERS, workspace=kws)
+
+        def do_km_warm():
+            sparse_attn_kmeans_permutation(Q, PERM_C, PERM_WARM_ITERS, init=Mq, workspace=kws)
+            sparse_attn_kmeans_permutation(K, PERM_C, PERM_WARM_ITERS, init=Mk, workspace=kws)
+
+        def do_gather():
+            sparse_attn_permute_rows(Q, pq, out=Qp)
+            sparse_attn_permute_rows(K, pk, out=Kp)
+            sparse_attn_permute_rows(V, pk, out=Vp)
+
+        def do_maskp():
+            sparse_attn_mask(Qp, Kp, bq, bk, k, p, out=outp, workspace=ws)
+
+        def do_fwdp():
+            sparse_attn_fwd(Qp, Kp, Vp, outp["cnt"], outp["idx"], bq, bk, out=Op)
+
+        def do_scatter():
+            sparse_attn_permute_rows(Op, pq, inverse=True, out=O_tok)
+        perm_fns = [do_km_warm, do_gather, do_maskp, do_fwdp, do_scatter]
+        for fn in perm_fns:
+            fn()
+        cold_ms, = loop_time([do_km_cold], 2)
+        warm_ms, gat_ms, maskp_ms, fwdp_ms, sca_ms = loop_time(perm_fns, max(5, min(args.steps, 10)))
+        check_device_error(dev)
+        flp, tilesp = kept_flops(outp["cnt"], outp["idx"], N, d, bq, bk)
+        # The assignment's fp32 operations (subtract, multiply, add per token,
+        # centroid and channel) against the non-fused fp32 issue rate.
+        assign_ops = 3.0 * B * H * N * PERM_C * d
+        alu_peak = 148 * 128 * 1.965e9
+        warm_assign_ms = 2 * (PERM_WARM_ITERS + 1) * assign_ops / alu_peak * 1e3
+        gather_bytes = 3 * 4.0 * B * H * N * d          # Q, K, V rows read and written once, bf16
+        perm_entry = {
+            "clusters_q": PERM_C, "clusters_k": PERM_C, "iters_cold": PERM_COLD_ITERS,
+            "iters_warm": PERM_WARM_ITERS,
+            "ms_per_call": {"kmeans_qk_cold": cold_ms, "kmeans_qk_warm": warm_ms, "gather_qkv": gat_ms,
+                            "mask": maskp_ms, "fwd": fwdp_ms, "scatter_o": sca_ms,
+                            "path_warm": warm_ms + gat_ms + maskp_ms + fwdp_ms + sca_ms},
+            "block_sparsity": 1.0 - tilesp / float(B * H * n_q * n_k),
+            "block_sparsity_unpermuted": sparsity,
+            "kept_tile_tflops_fwd": flp / (fwdp_ms * 1e-3) / 1e12,
+            "kmeans_warm_alu_frac": warm_assign_ms / warm_ms,
+            "gather_qkv_hbm_frac": gather_bytes / (gat_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "counting": "kmeans_warm_alu_frac: the assignments' 3 N C d fp32 operations per head "
+                        "and round (Q and K, iters + 1 assignments each) at 148 SMs x 128 lanes x "
+                        "1.965 GHz, over the whole warm k-means time (updates and sorts included); "
+                        "gather: 2 x 2 x N d bytes per head and tensor (bf16 read and write)",
+        }
         # End to end through the public host-buffer entry point (pinned host
         # Q, K, V in; O back in host memory): the library pipelines the copies
         # with the mask and attention by chunks of heads.
@@ -593,6 +664,7 @@ def run_ours(args):
                 "counted); bf16 gradients; fp8: per-block e4m3 Q and K, bf16 P V; sparse_linear: the linear "
                 "branch and the alpha mix given the sparse output (features, per-head state, kept tiles and "
                 "totals), its TFLOP/s counted on the kept tiles' products alone")),
+            "semantic_permutation": perm_entry,
             "e2e": {"value": fl / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2},
         }

@@ -456,6 +456,29 @@ def run_ours(args):
         fwd95_ms = statistics.fmean(e[1].elapsed_time(e[2]) for e in ev95)
         check_device_error(dev)
         s95 = 1.0 - tiles95 / float(B * H * n_q * n_k)
+        # The single-launch path (mask and attention in one cooperative kernel)
+        # at both points, timed the same way.
+        from block_sparse_attention_row_b200 import fused_workspace_bytes, sparse_attn_fused
+        fused_ms = {}
+        fws_n = fused_workspace_bytes(B, H, N, d, bq, bk)
+        if fws_n:
+            fws = torch.empty(fws_n, dtype=torch.uint8, device=dev)
+            fout = {"O": torch.empty_like(O), "cnt": torch.empty_like(out["cnt"]), "idx": torch.empty_like(out["idx"])}
+            for tag, (kk, pp) in (("config", (k, p)), ("sparsity_95_point", (k, 0.0))):
+                def do_fused():
+                    sparse_attn_fused(Q, K, V, bq, bk, kk, pp, out=fout, workspace=fws)
+                for _ in range(3):
+                    do_fused()
+                torch.cuda.synchronize()
+                reps = max(args.steps, 20) if tag == "sparsity_95_point" else args.steps
+                evf = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+                for i in range(reps):
+                    evf[i].record(stream)
+                    do_fused()
+                evf[reps].record(stream)
+                torch.cuda.synchronize()
+                fused_ms[tag] = statistics.fmean(evf[i].elapsed_time(evf[i + 1]) for i in range(reps))
+            check_device_error(dev)
         # Backward pass and the FP8 forward, each timed in its own loop of
         # back-to-back launches with events between them (as above), at the
         # workload's (k, p) and at the 95% point.
@@ -639,6 +662,11 @@ def run_ours(args):
                 "fwd_only": dense_ms / fwd_ms, "mask_plus_fwd": dense_ms / (mask_ms + fwd_ms),
                 "ideal_1_over_1_minus_s": 1.0 / max(1e-9, 1.0 - sparsity)},
             "dense_tflops": None if dense_ms is None else dense_flops(B, H, N, d) / (dense_ms * 1e-3) / 1e12,
+            "single_launch": None if not fused_ms else {
+                "ms_per_call": fused_ms,
+                "vs_mask_plus_fwd": {"config": mask_ms + fwd_ms, "sparsity_95_point": mask95_ms + fwd95_ms},
+                "kernel": "sparse_attn_fwd_kernel (cooperative: pooling, grid barrier, scores and selection, "
+                          "grid barrier, attention)"},
             "sparsity_95_point": {
                 "k": k, "p": 0.0, "block_sparsity": s95, "kept_tiles": tiles95, "steps": steps95,
                 "ms_per_call": {"mask": mask95_ms, "fwd": fwd95_ms},

@@ -28,6 +28,7 @@ EXPORTED = ("sparse_attn_mask_workspace_bytes", "sparse_attn_mask", "sparse_attn
             "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8",
             "sparse_attn_sparse_linear_workspace_bytes", "sparse_attn_sparse_linear",
             "sparse_attn_kmeans_workspace_bytes", "sparse_attn_kmeans_permutation", "sparse_attn_permute_rows",
+            "sparse_attn_fused_workspace_bytes", "sparse_attn_fused",
             "sparse_attn_fwd", "sparse_attn_fwd_dense", "sparse_attn_host_workspace_bytes",
             "sparse_attn_host", "sparse_attn_check_device_error",
             "sparse_attn_last_error", "sparse_attn_version", "sparse_attn_test_fwd_withheld_copy")
@@ -88,6 +89,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.sparse_attn_sparse_linear.argtypes = [sp, vp, vp, vp, i32p, i32p, vp, f32p, vp, ctypes.c_int, vp,
                                                   ctypes.c_size_t, vp]
         lib.sparse_attn_sparse_linear.restype = ctypes.c_int
+        lib.sparse_attn_fused_workspace_bytes.argtypes = [sp]
+        lib.sparse_attn_fused_workspace_bytes.restype = ctypes.c_size_t
+        lib.sparse_attn_fused.argtypes = [sp, vp, vp, vp, ctypes.c_double, ctypes.c_double, i32p, i32p, vp,
+                                          ctypes.c_int, f32p, vp, ctypes.c_size_t, vp]
+        lib.sparse_attn_fused.restype = ctypes.c_int
         lib.sparse_attn_kmeans_workspace_bytes.argtypes = [sp, ctypes.c_int]
         lib.sparse_attn_kmeans_workspace_bytes.restype = ctypes.c_size_t
         lib.sparse_attn_kmeans_permutation.argtypes = [sp, vp, ctypes.c_int, ctypes.c_int, f32p, i32p, i32p, f32p,
@@ -422,6 +428,47 @@ def sparse_attn_sparse_linear(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                        _stream(dev, stream))
     _check("sparse_attn_sparse_linear", st)
     return O
+
+
+def fused_workspace_bytes(B, H, N, d, bq, bk) -> int:
+    shape = make_shape(B, H, N, d, bq, bk)
+    return int(load_library().sparse_attn_fused_workspace_bytes(ctypes.byref(shape)))
+
+
+def sparse_attn_fused(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bq: int, bk: int, k: float, p: float, *,
+                      out_dtype=torch.bfloat16, want_lse: bool = False, out: Optional[dict] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Mask and attention in one cooperative kernel launch (SpargeAttention2
+    §2C). Returns {"O", "cnt", "idx"} (and "lse"), bit-equal to
+    sparse_attn_mask followed by sparse_attn_fwd."""
+    _check_qkv(Q, K, V)
+    B, H, N, d = Q.shape
+    n_q, n_k = num_blocks(N, bq, bk)
+    dev = Q.device
+    out = {} if out is None else out
+    for key, shp, dt in (("cnt", (B, H, n_q), torch.int32), ("idx", (B, H, n_q, n_k), torch.int32),
+                         ("lse", (B, H, N), torch.float32)):
+        if key == "lse" and not want_lse:
+            continue
+        if key not in out:
+            out[key] = torch.empty(shp, dtype=dt, device=dev)
+        t = out[key]
+        if t.dtype != dt or tuple(t.shape) != shp or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"out[{key!r}] must be a contiguous {dt} tensor {shp} on {dev}")
+    out["O"] = _out_tensor(Q, out.get("O"), out_dtype)
+    lib = load_library()
+    shape = make_shape(B, H, N, d, bq, bk)
+    nbytes = int(lib.sparse_attn_fused_workspace_bytes(ctypes.byref(shape)))
+    if nbytes == 0:
+        raise ValueError("unsupported shape for the single-launch path (n_k above its shared-memory limit?)")
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = lib.sparse_attn_fused(ctypes.byref(shape), _ptr(Q), _ptr(K), _ptr(V), float(k), float(p), _ptr(out["cnt"]),
+                               _ptr(out["idx"]), _ptr(out["O"]), SA_F32 if out_dtype == torch.float32 else SA_BF16,
+                               _ptr(out.get("lse")), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(dev, stream))
+    _check("sparse_attn_fused", st)
+    return out
 
 
 def kmeans_workspace_bytes(B, H, N, d, C, bq: int = 64, bk: int = 64) -> int:

@@ -43,6 +43,7 @@
 #include <cstdint>
 
 #include "sa_ptx.cuh"
+#include "sa_mask_kernels.cuh"
 
 namespace sa {
 namespace attn {
@@ -76,7 +77,8 @@ constexpr int MAX_CH = 4;
 // Where a bounded wait gave up (reported in the device error record).
 enum WaitSite : unsigned int {
     W_CH_EMPTY = 0xE001, W_Q = 0xE002, W_CH_FULL = 0xE003, W_P_FULL = 0xE004,
-    W_S_FULL = 0xE005, W_O_FULL = 0xE006, W_Q_EMPTY = 0xE007, W_LOCK = 0xE008, W_STG = 0xE009
+    W_S_FULL = 0xE005, W_O_FULL = 0xE006, W_Q_EMPTY = 0xE007, W_LOCK = 0xE008, W_STG = 0xE009,
+    W_GRID_POOL = 0xE00A, W_GRID_SELECT = 0xE00B
 };
 
 // FP8: Q and K are e4m3 codes (one byte per element, 128 channels per
@@ -140,6 +142,18 @@ struct Params {
     // FP8 path: per-block scales of the Q and K codes (null otherwise).
     const float* q_scale;   // [BH * n_q]
     const float* k_scale;   // [BH * n_k]
+    // Single-launch path only: the mask phases' inputs and outputs. cnt and
+    // idx above are then the buffers these phases write (cnt_w, idx_w).
+    const void* q_in;       // bf16 Q, K [BH, N, D]
+    const void* k_in;
+    float* qbar;            // [BH * n_q, D] block means (workspace)
+    float* kbar;            // [BH * n_k, D]
+    unsigned int* grid_ctr; // grid-barrier counter, zeroed before the launch
+    int32_t* cnt_w;
+    int32_t* idx_w;
+    int BH, bq, kc;
+    double p;
+    float score_scale;      // 1/sqrt(d)
 };
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr) {
@@ -247,10 +261,19 @@ __device__ __forceinline__ void umma_ts_batch8(uint32_t d, uint32_t a_tmem, cons
         : "memory");
 }
 
+// The lists are read through the read-only path, except on the single-launch
+// path (CG), where this launch wrote them: there they are read through L2.
+template <bool CG>
+__device__ __forceinline__ int ld_list(const int32_t* p) {
+    if constexpr (CG) return __ldcg(p);
+    else return __ldg(p);
+}
+
 // Kept-block count of a row as stored (loaded a row ahead, checked at use, so
 // that the load's latency is not waited for until then).
+template <bool CG>
 __device__ __forceinline__ int raw_count(const Params& prm, int r) {
-    return prm.dense ? prm.n_k : __ldg(prm.cnt + r);
+    return prm.dense ? prm.n_k : ld_list<CG>(prm.cnt + r);
 }
 // A count range-checked (a bad count is recorded and clamped).
 __device__ __forceinline__ int checked_count(const Params& prm, int c) {
@@ -262,16 +285,18 @@ __device__ __forceinline__ int checked_count(const Params& prm, int c) {
 }
 
 // Index-list entry e of row r for this lane, -1 past the row's count.
+template <bool CG>
 __device__ __forceinline__ int list_entry(const Params& prm, int r, int cnt, int e) {
     if (e >= cnt) return -1;
-    return prm.dense ? e : __ldg(prm.idx + (size_t)r * prm.n_k + e);
+    return prm.dense ? e : ld_list<CG>(prm.idx + (size_t)r * prm.n_k + e);
 }
 
 // Index-list entry e of row r without the count check (-1 past n_k): loaded a
 // row ahead, before the row's count is known, and masked with it at use.
+template <bool CG>
 __device__ __forceinline__ int raw_entry(const Params& prm, int r, int e) {
     if (r >= prm.rows || e >= prm.n_k) return -1;
-    return prm.dense ? e : __ldg(prm.idx + (size_t)r * prm.n_k + e);
+    return prm.dense ? e : ld_list<CG>(prm.idx + (size_t)r * prm.n_k + e);
 }
 
 // Ticket lock that hands the tensor pipe to one issuer's batch at a time.
@@ -298,7 +323,7 @@ __device__ __forceinline__ void issue_release(Ctrl& C, int ticket) {
     *reinterpret_cast<volatile int*>(&C.ticket_serving) = ticket + 1;
 }
 
-template <int D, int BQ, bool FP8 = false>
+template <int D, int BQ, bool FP8 = false, bool FUSED = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -347,7 +372,25 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     const uint32_t tmem = C.tmem_base;
     const uint64_t lim = prm.wait_limit_ns;
 
-    if (warp >= 8) {
+    if constexpr (FUSED) {
+        // The mask, in this launch (cooperative: every CTA is resident): the
+        // block means, a grid barrier, the scores and kept lists of every row,
+        // a grid barrier; then the attention below reads the lists. Shared
+        // memory below the control block serves as the phases' scratch.
+        sa::mask::fused_pool_phase<D>(static_cast<const __nv_bfloat16*>(prm.q_in),
+                                      static_cast<const __nv_bfloat16*>(prm.k_in), prm.qbar, prm.kbar, prm.BH,
+                                      prm.N, prm.bq, BK, prm.n_q, n_k, reinterpret_cast<float*>(smem));
+        if (sa::mask::grid_barrier(prm.grid_ctr, gridDim.x, lim, abort_flag, W_GRID_POOL))
+            sa::mask::fused_select_phase<D>(prm.qbar, prm.kbar, prm.BH, prm.n_q, n_k, prm.score_scale, prm.kc,
+                                            prm.p, prm.cnt_w, prm.idx_w, smem);
+        // The scratch is rewritten by TMA and read by the MMAs (async proxy).
+        fence_proxy_async_smem();
+        sa::mask::grid_barrier(prm.grid_ctr, 2 * gridDim.x, lim, abort_flag, W_GRID_SELECT);
+    }
+
+    if (FUSED && *abort_flag) {
+        // A grid barrier ran out: no attention (nothing was issued).
+    } else if (warp >= 8) {
       // Control warpgroup: producers and MMA issuers.
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(CTRL_REGS));
       if (warp == PRODUCER_WARP0 || warp == PRODUCER_WARP1) {
@@ -365,15 +408,15 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         bool ok = true;
         // The next row's count and first 64 index entries are loaded a row ahead.
         const int r_first = blockIdx.x * NSLOT + s;
-        int cnt_next = r_first < prm.rows ? raw_count(prm, r_first) : 0;
-        int raw0_next = raw_entry(prm, r_first, lane), raw1_next = raw_entry(prm, r_first, 32 + lane);
+        int cnt_next = r_first < prm.rows ? raw_count<FUSED>(prm, r_first) : 0;
+        int raw0_next = raw_entry<FUSED>(prm, r_first, lane), raw1_next = raw_entry<FUSED>(prm, r_first, 32 + lane);
         for (int r = r_first; ok && r < prm.rows; r += P) {
             const int cnt = checked_count(prm, cnt_next);
             const int raw0 = raw0_next, raw1 = raw1_next;
             if (r + P < prm.rows) {
-                cnt_next = raw_count(prm, r + P);
-                raw0_next = raw_entry(prm, r + P, lane);
-                raw1_next = raw_entry(prm, r + P, 32 + lane);
+                cnt_next = raw_count<FUSED>(prm, r + P);
+                raw0_next = raw_entry<FUSED>(prm, r + P, lane);
+                raw1_next = raw_entry<FUSED>(prm, r + P, 32 + lane);
             }
             const int nt = (cnt + 1) / 2;
             if (nt == 0) continue;
@@ -398,7 +441,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const int e0 = 2 * t;
                 if (e0 > 0 && (e0 & 31) == 0) {
                     window = window_next;
-                    window_next = list_entry(prm, r, cnt, e0 + 32 + lane);
+                    window_next = list_entry<FUSED>(prm, r, cnt, e0 + 32 + lane);
                 }
                 int j0 = __shfl_sync(0xFFFFFFFFu, window, e0 & 31);
                 int j1 = __shfl_sync(0xFFFFFFFFu, window, (e0 + 1) & 31);
@@ -484,10 +527,10 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             int k = 0, g = 0, kq = 0, ticket = 0;
             bool ok = true;
             const int r_first = blockIdx.x * NSLOT + s;
-            int cnt_next = r_first < prm.rows ? raw_count(prm, r_first) : 0;   // a row ahead
+            int cnt_next = r_first < prm.rows ? raw_count<FUSED>(prm, r_first) : 0;   // a row ahead
             for (int r = r_first; ok && r < prm.rows; r += P) {
                 const int nt = (checked_count(prm, cnt_next) + 1) / 2;
-                if (r + P < prm.rows) cnt_next = raw_count(prm, r + P);
+                if (r + P < prm.rows) cnt_next = raw_count<FUSED>(prm, r + P);
                 if (nt == 0) continue;
                 if (!mbar_wait_bounded(&B.q_full, kq & 1, abort_flag, W_Q, lim) || !wait_chunk(k)) {
                     ok = false;
@@ -562,15 +605,15 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         bool ok = true;
         // The next row's count and first 64 index entries are loaded a row ahead.
         const int r_first = blockIdx.x * NSLOT + s;
-        int cnt_next = r_first < prm.rows ? raw_count(prm, r_first) : 0;
-        int raw0_next = raw_entry(prm, r_first, lane), raw1_next = raw_entry(prm, r_first, 32 + lane);
+        int cnt_next = r_first < prm.rows ? raw_count<FUSED>(prm, r_first) : 0;
+        int raw0_next = raw_entry<FUSED>(prm, r_first, lane), raw1_next = raw_entry<FUSED>(prm, r_first, 32 + lane);
         for (int r = r_first; ok && r < prm.rows; r += P) {
             const int cnt = checked_count(prm, cnt_next);
             const int raw0 = raw0_next, raw1 = raw1_next;
             if (r + P < prm.rows) {
-                cnt_next = raw_count(prm, r + P);
-                raw0_next = raw_entry(prm, r + P, lane);
-                raw1_next = raw_entry(prm, r + P, 32 + lane);
+                cnt_next = raw_count<FUSED>(prm, r + P);
+                raw0_next = raw_entry<FUSED>(prm, r + P, lane);
+                raw1_next = raw_entry<FUSED>(prm, r + P, 32 + lane);
             }
             const int nt = (cnt + 1) / 2;
             const int bh = r / prm.n_q, qb = r % prm.n_q;
@@ -589,7 +632,7 @@ sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 const int e0 = 2 * t;
                 if (e0 > 0 && (e0 & 31) == 0) {
                     window = window_next;
-                    window_next = list_entry(prm, r, cnt, e0 + 32 + lane);
+                    window_next = list_entry<FUSED>(prm, r, cnt, e0 + 32 + lane);
                 }
                 const int j0 = checked(__shfl_sync(0xFFFFFFFFu, window, e0 & 31));
                 const int j1 = (e0 + 1 < cnt) ? checked(__shfl_sync(0xFFFFFFFFu, window, (e0 + 1) & 31)) : -1;

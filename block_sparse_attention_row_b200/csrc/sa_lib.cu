@@ -229,10 +229,20 @@ struct Fp8Scales {
     const float* k = nullptr;
 };
 
-template <int D, int BQ, bool FP8 = false>
+// The single-launch path's extra arguments (the mask phases).
+struct FusedArgs {
+    float* qbar = nullptr;
+    float* kbar = nullptr;
+    unsigned int* grid_ctr = nullptr;
+    int kc = 0;
+    double p = 0.0;
+};
+
+template <int D, int BQ, bool FP8 = false, bool FUSED = false>
 sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void* V, const int32_t* cnt,
                         const int32_t* idx, void* O, bool out_f32, float* lse, bool dense,
-                        cudaStream_t st, const AttnTestKnobs& knobs, const Fp8Scales& sc = Fp8Scales()) {
+                        cudaStream_t st, const AttnTestKnobs& knobs, const Fp8Scales& sc = Fp8Scales(),
+                        const FusedArgs& fz = FusedArgs()) {
     using L = sa::attn::Layout<D, FP8>;
     CUtensorMap mq, mk, mv, mo;
     sa_status s;
@@ -248,7 +258,7 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
     // fp32 output is written directly (the map is then unused).
     if (out_f32) mo = mq;
     else if ((s = make_map(&mo, O, g, BQ)) != SA_OK) return s;
-    auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ, FP8>;
+    auto kern = sa::attn::sparse_attn_fwd_kernel<D, BQ, FP8, FUSED>;
     if ((s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::DYN_BYTES),
                         "sparse_attn_fwd_kernel shared-memory attribute")) != SA_OK)
         return s;
@@ -275,9 +285,39 @@ sa_status launch_attn_t(const Dims& g, const void* Q, const void* K, const void*
     prm.withhold_first_k = knobs.withhold_first_k;
     prm.q_scale = sc.q;
     prm.k_scale = sc.k;
+    prm.q_in = Q;
+    prm.k_in = K;
+    prm.qbar = fz.qbar;
+    prm.kbar = fz.kbar;
+    prm.grid_ctr = fz.grid_ctr;
+    prm.cnt_w = const_cast<int32_t*>(cnt);
+    prm.idx_w = const_cast<int32_t*>(idx);
+    prm.BH = g.BH;
+    prm.bq = g.bq;
+    prm.kc = fz.kc;
+    prm.p = fz.p;
+    prm.score_scale = (float)(1.0 / std::sqrt((double)D));
     // Persistent: one CTA per multiprocessor (fewer when there are fewer row pairs).
     const int pairs = (prm.rows + sa::attn::NSLOT - 1) / sa::attn::NSLOT;
     const int grid = pairs < sm_count() ? pairs : sm_count();
+    if constexpr (FUSED) {
+        // Cooperative launch: the grid barriers need every CTA resident at
+        // once, which the launch guarantees (or refuses).
+        if ((s = cuda_check(cudaMemsetAsync(fz.grid_ctr, 0, sizeof(unsigned int), st), "zero the grid counter")) !=
+            SA_OK)
+            return s;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(sa::attn::NUM_THREADS);
+        cfg.dynamicSmemBytes = L::DYN_BYTES;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cuda_check(cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, prm), "single-launch kernel launch");
+    }
     kern<<<grid, sa::attn::NUM_THREADS, L::DYN_BYTES, st>>>(mq, mk, mv, mo, prm);
     return cuda_check(cudaGetLastError(), "sparse_attn_fwd_kernel launch");
 }
@@ -509,6 +549,32 @@ sa_status launch_sparse_linear(const Dims& g, const void* Q, const void* K, cons
     return cuda_check(cudaGetLastError(), "sparse_linear_kernel launch");
 }
 
+// ------------------------------------------------- single-launch path
+// Workspace: the block means (fp32, as the mask's) and the grid counter.
+struct FusedLayout {
+    size_t qbar, kbar, ctr, total;
+};
+
+FusedLayout fused_layout(const Dims& g) {
+    FusedLayout w;
+    w.qbar = 0;
+    w.kbar = round256((size_t)g.BH * g.n_q * g.d * sizeof(float));
+    w.ctr = w.kbar + round256((size_t)g.BH * g.n_k * g.d * sizeof(float));
+    w.total = w.ctr + 256;
+    return w;
+}
+
+// The selection phase keeps a tile of rows' logits and masses in the
+// attention kernel's shared memory (below its control block).
+sa_status check_fused_shape(const Dims& g) {
+    const size_t room = g.d == 128 ? (size_t)sa::attn::Layout<128>::OFF_CTRL : (size_t)sa::attn::Layout<64>::OFF_CTRL;
+    const size_t need = sa::mask::fused_select_smem(g.d, g.n_k);
+    if (need > room)
+        return fail(SA_ERR_UNSUPPORTED, "single-launch path: n_k=%d needs %zu bytes of shared memory for its "
+                    "selection phase, %zu available (use sparse_attn_mask + sparse_attn_fwd)", g.n_k, need, room);
+    return SA_OK;
+}
+
 // ------------------------------------------- semantic-aware permutation
 constexpr int KM_MAX_C = 8192;
 constexpr int KM_MAX_ITERS = 100;
@@ -551,6 +617,47 @@ sa_status launch_kmeans(const Dims& g, const void* X, int C, int iters, const fl
 }  // namespace
 
 extern "C" {
+
+size_t sparse_attn_fused_workspace_bytes(const sa_shape* shape) {
+    Dims g;
+    if (check_shape(shape, g) != SA_OK || check_fused_shape(g) != SA_OK) return 0;
+    return fused_layout(g).total;
+}
+
+sa_status sparse_attn_fused(const sa_shape* shape, const void* Q, const void* K, const void* V, double k, double p,
+                            int32_t* cnt, int32_t* idx, void* O, int o_dtype, float* lse_or_null, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    Dims g;
+    sa_status s;
+    if ((s = check_fwd_args(shape, Q, K, V, cnt, idx, O, o_dtype, lse_or_null, g)) != SA_OK) return s;
+    if ((s = check_kp(k, p)) != SA_OK) return s;
+    if ((s = check_fused_shape(g)) != SA_OK) return s;
+    if (!workspace) return fail(SA_ERR_INVALID_ARG, "NULL workspace");
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(SA_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+    const FusedLayout w = fused_layout(g);
+    if (workspace_bytes < w.total)
+        return fail(SA_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", workspace_bytes, w.total);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    FusedArgs fa;
+    fa.qbar = reinterpret_cast<float*>(ws + w.qbar);
+    fa.kbar = reinterpret_cast<float*>(ws + w.kbar);
+    fa.grid_ctr = reinterpret_cast<unsigned int*>(ws + w.ctr);
+    fa.kc = topk_count(k, g.n_k);
+    fa.p = p;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool f32 = o_dtype == SA_F32;
+    const AttnTestKnobs kn;
+    if (g.d == 128 && g.bq == 128)
+        s = launch_attn_t<128, 128, false, true>(g, Q, K, V, cnt, idx, O, f32, lse_or_null, false, st, kn, {}, fa);
+    else if (g.d == 128)
+        s = launch_attn_t<128, 64, false, true>(g, Q, K, V, cnt, idx, O, f32, lse_or_null, false, st, kn, {}, fa);
+    else if (g.bq == 128)
+        s = launch_attn_t<64, 128, false, true>(g, Q, K, V, cnt, idx, O, f32, lse_or_null, false, st, kn, {}, fa);
+    else
+        s = launch_attn_t<64, 64, false, true>(g, Q, K, V, cnt, idx, O, f32, lse_or_null, false, st, kn, {}, fa);
+    if (s != SA_OK) return s;
+    return ok();
+}
 
 size_t sparse_attn_kmeans_workspace_bytes(const sa_shape* shape, int C) {
     Dims g;

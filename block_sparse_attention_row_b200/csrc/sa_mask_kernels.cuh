@@ -27,6 +27,46 @@ namespace mask {
 
 constexpr int POOL_THREADS = 128;
 
+// Mean of the valid rows of one block of X (`valid` token rows of D bf16
+// channels from `src`), computed by the POOL_THREADS threads of a group
+// (tid = 0 .. POOL_THREADS-1) through `red` ([POOL_THREADS / (D / 8)][D]
+// floats of shared memory), `sync` being the group's barrier. Each thread
+// sums its 16-byte column chunk over the rows tid / (D / 8), + RG, ... in
+// order; the partial sums are then added in group order and divided by
+// `valid`. Used by pool_kernel and by the single-launch path, so both give
+// the same bits.
+template <int D, typename Sync>
+__device__ __forceinline__ void pool_block(const __nv_bfloat16* __restrict__ src_rows, float* __restrict__ out,
+                                           int valid, int tid, float* red, Sync sync) {
+    constexpr int CG = D / 8;              // 16-byte chunks per token row
+    constexpr int RG = POOL_THREADS / CG;  // token rows read in parallel
+    const uint4* src = reinterpret_cast<const uint4*>(src_rows);
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 8
+    for (int r = rg; r < valid; r += RG) {
+        const uint4 v = __ldg(src + (size_t)r * CG + cg);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[2 * e] += __uint_as_float(w[e] << 16);
+            acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rg * D + cg * 8 + e] = acc[e];
+    sync();
+    for (int c = tid; c < D; c += POOL_THREADS) {
+        float s = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) s += red[g * D + c];
+        out[c] = s / (float)valid;
+    }
+}
+
 // Mean of the valid tokens of one query block or key block. blockIdx.x in
 // [0, n_q) pools a Q block, [n_q, n_q + n_k) a K block; blockIdx.y = b*H + h.
 template <int D>
@@ -34,10 +74,7 @@ __global__ void __launch_bounds__(POOL_THREADS)
 pool_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
             float* __restrict__ Qbar, float* __restrict__ Kbar, int N, int bq, int bk, int n_q,
             int n_k) {
-    constexpr int CG = D / 8;              // 16-byte chunks per token row
-    constexpr int RG = POOL_THREADS / CG;  // token rows read in parallel
-    __shared__ float red[RG][D];
-
+    __shared__ float red[(POOL_THREADS / (D / 8)) * D];
     const int bh = blockIdx.y;
     int blk = blockIdx.x;
     const __nv_bfloat16* X;
@@ -55,32 +92,7 @@ pool_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict
     }
     const int lo = blk * bs;
     const int valid = min(N - lo, bs);
-    const uint4* src = reinterpret_cast<const uint4*>(X + ((size_t)bh * N + lo) * D);
-    const int cg = threadIdx.x % CG;
-    const int rg = threadIdx.x / CG;
-
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 8
-    for (int r = rg; r < valid; r += RG) {
-        const uint4 v = __ldg(src + (size_t)r * CG + cg);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            acc[2 * e] += __uint_as_float(w[e] << 16);
-            acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[rg][cg * 8 + e] = acc[e];
-    __syncthreads();
-    for (int c = threadIdx.x; c < D; c += POOL_THREADS) {
-        float s = 0.f;
-#pragma unroll
-        for (int g = 0; g < RG; ++g) s += red[g][c];
-        out[c] = s / (float)valid;
-    }
+    pool_block<D>(X + ((size_t)bh * N + lo) * D, out, valid, threadIdx.x, red, [] { __syncthreads(); });
 }
 
 // logits[bh*n_q + i][j] = scale * sum_c Qbar[bh,i,c] * Kbar[bh,j,c], fp32.
@@ -294,8 +306,9 @@ inline int select_warps_per_cta(int n_k) {
     return w < 1 ? 1 : (w > SEL_MAX_WARPS ? SEL_MAX_WARPS : w);
 }
 
-// One warp per score row. The kept set is the first L entries of the order
-// "score descending, then index ascending", L = max(kc, m_p):
+// The selection of one score row by one warp. The kept set is the first L
+// entries of the order "score descending, then index ascending",
+// L = max(kc, m_p):
 //   kc  = number of Top-k blocks (computed on the host);
 //   m_p = shortest prefix whose fixed-point mass reaches T = ceil(p * W).
 // m_p comes from the mass boundary v (entries above v, then as many of the
@@ -303,20 +316,13 @@ inline int select_warps_per_cta(int n_k) {
 // count boundary of kc is searched the same way. The kept indices are then
 // written in ascending order, ties at the boundary taken by lower index.
 // The result equals the prefix of a full sort bit for bit.
+// src: the row's logits (FROM_LOGITS: softmax taken here) or scores; bits:
+// n_k words of scratch, which may be src itself (each lane rewrites only the
+// entries it read); masses: n_k 8-byte words of scratch. Returns L.
 template <bool FROM_LOGITS>
-__global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
-select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
-              int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
-              float* __restrict__ P_out) {
-    extern __shared__ __align__(8) unsigned char sel_smem[];
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int wpc = blockDim.x / 32;
-    const long long row = (long long)blockIdx.x * wpc + warp;
-    if (row >= n_rows) return;
-    uint32_t* bits = reinterpret_cast<uint32_t*>(sel_smem + (size_t)warp * select_row_bytes(n_k));
-    uint64_t* masses = reinterpret_cast<uint64_t*>(bits + ((n_k + 1) & ~1));
-    const float* src = in + (size_t)row * ld_in;
-
+__device__ int select_row(const float* src, int n_k, int kc, double p, uint32_t* bits, uint64_t* masses,
+                          int32_t* __restrict__ idx_row, uint8_t* __restrict__ mask_row, float* __restrict__ P_row,
+                          int lane) {
     if (FROM_LOGITS) {
         float mx = -INFINITY;
         for (int j = lane; j < n_k; j += 32) mx = fmaxf(mx, src[j]);
@@ -338,7 +344,7 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
         for (int j = lane; j < n_k; j += 32) {
             const float pj = fminf(__uint_as_float(bits[j]) * inv, 1.0f);
             bits[j] = __float_as_uint(pj);
-            if (P_out) P_out[(size_t)row * n_k + j] = pj;
+            if (P_row) P_row[j] = pj;
         }
     } else {
         bool bad = false;
@@ -383,8 +389,6 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
     }
     L = min(L, n_k);
 
-    int32_t* idx_row = idx + (size_t)row * n_k;
-    uint8_t* mask_row = mask ? mask + (size_t)row * n_k : nullptr;
     if (L == n_k) {
         for (int j = lane; j < n_k; j += 32) {
             idx_row[j] = j;
@@ -416,7 +420,177 @@ select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int 
             kept_before += __popc(keep_ballot);
         }
     }
+    return L;
+}
+
+// One warp per score row (select_row above), rows in shared memory.
+template <bool FROM_LOGITS>
+__global__ void __launch_bounds__(SEL_MAX_WARPS * 32)
+select_kernel(const float* __restrict__ in, int ld_in, int n_rows, int n_k, int kc, double p,
+              int32_t* __restrict__ cnt, int32_t* __restrict__ idx, uint8_t* __restrict__ mask,
+              float* __restrict__ P_out) {
+    extern __shared__ __align__(8) unsigned char sel_smem[];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int wpc = blockDim.x / 32;
+    const long long row = (long long)blockIdx.x * wpc + warp;
+    if (row >= n_rows) return;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(sel_smem + (size_t)warp * select_row_bytes(n_k));
+    uint64_t* masses = reinterpret_cast<uint64_t*>(bits + ((n_k + 1) & ~1));
+    const int L = select_row<FROM_LOGITS>(in + (size_t)row * ld_in, n_k, kc, p, bits, masses,
+                                          idx + (size_t)row * n_k, mask ? mask + (size_t)row * n_k : nullptr,
+                                          P_out ? P_out + (size_t)row * n_k : nullptr, lane);
     if (lane == 0) cnt[row] = L;
+}
+
+// ------------------------------------------- single-launch mask phases
+// The mask steps run inside the attention kernel's launch (all of its
+// threads, before they take their attention roles), separated by grid
+// barriers. Each phase computes exactly what pool_kernel, score_kernel and
+// select_kernel compute, with the same per-element operation order, so the
+// block lists are identical to the three-launch path's.
+
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid barrier of a cooperative launch: every CTA adds one to *ctr and waits
+// until it reaches `target` (CTA count times the barrier's ordinal; the
+// counter is zeroed before the launch). The wait is bounded: past `lim` ns
+// the CTA records SA_STATUS_TIMEOUT with `site`, sets *abort_flag and goes
+// on; a CTA that has given up before arrives without waiting. Returns false
+// if this CTA has given up (now or earlier).
+__device__ __forceinline__ bool grid_barrier(unsigned int* ctr, unsigned int target, unsigned long long lim,
+                                             volatile int* abort_flag, unsigned int site) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);   // arrives even after giving up, so that no other CTA waits on this one
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t it = 0; *abort_flag == 0 && ld_acquire_gpu(ctr) < target; ++it) {
+            if ((it & 63u) == 63u && globaltimer_ns() - t0 > lim) {
+                record_error(SA_STATUS_TIMEOUT, site);
+                *abort_flag = 1;
+                break;
+            }
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return *abort_flag == 0;
+}
+
+// Phase A: the block means. Groups of POOL_THREADS threads (a warpgroup
+// each, named barrier 1 + group) take (head, block) items in turn, Q blocks
+// then K blocks of each head as pool_kernel's grid orders them.
+// red: the groups' reduction arrays, (blockDim.x / POOL_THREADS) x
+// (POOL_THREADS / (D / 8)) x D floats of shared memory.
+template <int D>
+__device__ void fused_pool_phase(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+                                 float* __restrict__ Qbar, float* __restrict__ Kbar, int BH, int N, int bq, int bk,
+                                 int n_q, int n_k, float* red_all) {
+    constexpr int RED = (POOL_THREADS / (D / 8)) * D;
+    const int grp = threadIdx.x / POOL_THREADS;
+    const int ngrp = blockDim.x / POOL_THREADS;
+    const int tid = threadIdx.x % POOL_THREADS;
+    float* red = red_all + grp * RED;
+    auto group_sync = [grp] { asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "n"(POOL_THREADS) : "memory"); };
+    const long long per_head = n_q + n_k;
+    const long long items = (long long)BH * per_head;
+    for (long long it = (long long)blockIdx.x * ngrp + grp; it < items; it += (long long)gridDim.x * ngrp) {
+        const int bh = (int)(it / per_head);
+        int blk = (int)(it % per_head);
+        const __nv_bfloat16* X;
+        float* out;
+        int bs;
+        if (blk < n_q) {
+            X = Q;
+            out = Qbar + ((size_t)bh * n_q + blk) * D;
+            bs = bq;
+        } else {
+            blk -= n_q;
+            X = K;
+            out = Kbar + ((size_t)bh * n_k + blk) * D;
+            bs = bk;
+        }
+        const int lo = blk * bs;
+        group_sync();   // the group's previous item has read red
+        pool_block<D>(X + ((size_t)bh * N + lo) * D, out, min(N - lo, bs), tid, red, group_sync);
+    }
+}
+
+// Rows of one phase-B item: one per warp of the attention kernel's CTA.
+constexpr int FUSED_ROWS = 12;
+
+// Shared memory phase B needs for a row length n_k (pooled query rows,
+// logits whose bits the selection overwrites in place, fixed-point masses).
+__host__ __device__ inline size_t fused_select_smem(int D, int n_k) {
+    const int ldk = (n_k + 3) & ~3;
+    return (size_t)FUSED_ROWS * D * 4 + (size_t)FUSED_ROWS * ldk * 4 + (size_t)FUSED_ROWS * n_k * 8;
+}
+
+// Phase B: scores and selection, an item being FUSED_ROWS query-block rows
+// of one head. The logits of the item's rows against every key block are
+// computed as score_kernel computes them (fp32 fused multiply-adds over the
+// channels in ascending order from 0, then times `scale`) into shared
+// memory; each warp then selects one row (select_row, as select_kernel) and
+// writes its kept list and count. Qbar and Kbar were written by other CTAs
+// before the grid barrier: they are read through L2 (ld.global.cg).
+template <int D>
+__device__ void fused_select_phase(const float* __restrict__ Qbar, const float* __restrict__ Kbar, int BH, int n_q,
+                                   int n_k, float scale, int kc, double p, int32_t* __restrict__ cnt,
+                                   int32_t* __restrict__ idx, uint8_t* smem) {
+    const int ldk = (n_k + 3) & ~3;
+    float* qs = reinterpret_cast<float*>(smem);                       // [FUSED_ROWS][D]
+    float* logit = qs + FUSED_ROWS * D;                               // [FUSED_ROWS][ldk]
+    uint64_t* masses = reinterpret_cast<uint64_t*>(logit + FUSED_ROWS * ldk);   // [FUSED_ROWS][n_k]
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nthr = blockDim.x;
+    const int tiles = (n_q + FUSED_ROWS - 1) / FUSED_ROWS;
+    const long long items = (long long)BH * tiles;
+    for (long long it = blockIdx.x; it < items; it += gridDim.x) {
+        const int bh = (int)(it / tiles);
+        const int i0 = (int)(it % tiles) * FUSED_ROWS;
+        const int nr = min(FUSED_ROWS, n_q - i0);
+        __syncthreads();   // the previous item is done with shared memory
+        for (int e = threadIdx.x; e < FUSED_ROWS * (D / 4); e += nthr) {
+            const int r = e / (D / 4), c4 = e % (D / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < nr) v = __ldcg(reinterpret_cast<const float4*>(Qbar + ((size_t)bh * n_q + i0 + r) * D) + c4);
+            reinterpret_cast<float4*>(qs + r * D)[c4] = v;
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < n_k; j += nthr) {
+            const float4* kr = reinterpret_cast<const float4*>(Kbar + ((size_t)bh * n_k + j) * D);
+            float acc[FUSED_ROWS];
+#pragma unroll
+            for (int r = 0; r < FUSED_ROWS; ++r) acc[r] = 0.f;
+#pragma unroll 4
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 kv = __ldcg(kr + c4);
+#pragma unroll
+                for (int r = 0; r < FUSED_ROWS; ++r) {
+                    const float4 qv = reinterpret_cast<const float4*>(qs + r * D)[c4];
+                    acc[r] = fmaf(qv.x, kv.x, acc[r]);
+                    acc[r] = fmaf(qv.y, kv.y, acc[r]);
+                    acc[r] = fmaf(qv.z, kv.z, acc[r]);
+                    acc[r] = fmaf(qv.w, kv.w, acc[r]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < FUSED_ROWS; ++r)
+                if (r < nr) logit[r * ldk + j] = acc[r] * scale;
+        }
+        __syncthreads();
+        if (warp < nr) {
+            float* row = logit + warp * ldk;
+            const size_t gr = (size_t)bh * n_q + i0 + warp;
+            const int L = select_row<true>(row, n_k, kc, p, reinterpret_cast<uint32_t*>(row),
+                                           masses + (size_t)warp * n_k, idx + gr * n_k, nullptr, nullptr, lane);
+            if (lane == 0) cnt[gr] = L;
+        }
+    }
 }
 
 }  // namespace mask

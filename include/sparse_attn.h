@@ -185,6 +185,44 @@ sa_status sparse_attn_fwd_fp8(const sa_shape* shape, const uint8_t* Q8, const ui
                               const int32_t* cnt, const int32_t* idx,
                               void* O, int o_dtype, float* lse_or_null, void* stream);
 
+/* Bytes of device workspace sparse_attn_fused needs for `shape`: the fp32
+ * block means of Q and K (4 * B*H*(n_q + n_k)*d, each part rounded up to
+ * 256) and a 256-byte grid-barrier counter. 0 on an invalid shape or one
+ * the single launch does not support (see below). */
+size_t sparse_attn_fused_workspace_bytes(const sa_shape* shape);
+
+/* Steps 1-4 in ONE kernel launch: "SpargeAttention2" §2C (Efficient Kernel
+ * Implementation) applies the block mask inside the FlashAttention-style
+ * kernel. The launch is cooperative (every CTA resident at once) and runs
+ * three phases separated by grid barriers: the block means of Q and K (as
+ * sparse_attn_mask step 1), then the scores and hybrid Top-k + Top-p lists
+ * of every query-block row (steps 2-3, a tile of 12 rows at a time in
+ * shared memory), then the block-sparse attention over those lists (step
+ * 4, as sparse_attn_fwd). Every phase takes the same operations in the same
+ * order as the separate entry points, so cnt, idx, O and lse are bit-equal
+ * to sparse_attn_mask followed by sparse_attn_fwd.
+ * Inputs:  Q, K, V bf16 [B,H,N,d]; k, p as for sparse_attn_mask.
+ * Outputs: cnt int32 [B,H,n_q] and idx int32 [B,H,n_q,n_k] (entries past
+ *          cnt unspecified), O [B,H,N,d] of type o_dtype, lse fp32 [B,H,N]
+ *          or NULL.
+ * workspace: device, sparse_attn_fused_workspace_bytes(shape) bytes,
+ *          256-byte aligned; workspace_bytes is checked against that size.
+ *          The grid counter in it is zeroed by a memset on `stream` before
+ *          the kernel, so calls that overlap on the GPU need separate
+ *          workspaces.
+ * Limits:  the selection phase holds 12 rows of n_k logits and fixed-point
+ *          masses in the attention kernel's shared memory: n_k <= 1549 for
+ *          d = 128 (N <= 99,136 tokens) and n_k <= 1344 for d = 64
+ *          (N <= 86,016); larger shapes get SA_ERR_UNSUPPORTED.
+ * Errors:  as sparse_attn_mask and sparse_attn_fwd; a grid barrier that
+ *          waits past the kernels' bound (4 s) is reported as SA_ERR_TIMEOUT
+ *          by sparse_attn_check_device_error and the attention phase is
+ *          skipped. */
+sa_status sparse_attn_fused(const sa_shape* shape, const void* Q, const void* K, const void* V,
+                            double k, double p, int32_t* cnt, int32_t* idx, void* O, int o_dtype,
+                            float* lse_or_null, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
 /* Bytes of device workspace sparse_attn_kmeans_permutation needs: the
  * cluster offsets, 4 * B*H*(C + 1) rounded up to 256. 0 on an invalid shape
  * or C. */

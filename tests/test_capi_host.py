@@ -249,3 +249,25 @@ def test_kmeans_binding_refuses_cpu_tensors():
         sparse_attn_kmeans_permutation(X, 4, 2)
     with pytest.raises(ValueError):
         sparse_attn_permute_rows(X, torch.zeros(1, 1, 64, dtype=torch.int32))
+
+
+def test_fused_host_validation(lib):
+    from block_sparse_attention_row_b200.capi import make_shape
+    a, z, ws = ctypes.c_void_p(16), ctypes.c_void_p(0), ctypes.c_void_p(256)
+    sh = ctypes.byref(make_shape(1, 2, 4096, 128, 128, 64))
+    need = lib.sparse_attn_fused_workspace_bytes(sh)
+    n_q, n_k = 32, 64
+    assert need == ((2 * n_q * 128 * 4 + 255) // 256) * 256 + ((2 * n_k * 128 * 4 + 255) // 256) * 256 + 256
+    # Rows longer than the selection phase's shared memory allows are refused:
+    # n_k <= 1549 for d = 128, n_k <= 1344 for d = 64.
+    for d, n_max in ((128, 1549), (64, 1344)):
+        assert lib.sparse_attn_fused_workspace_bytes(ctypes.byref(make_shape(1, 1, 64 * n_max, d, 128, 64))) > 0
+        assert lib.sparse_attn_fused_workspace_bytes(ctypes.byref(make_shape(1, 1, 64 * n_max + 1, d, 128, 64))) == 0
+    big = ctypes.byref(make_shape(1, 1, 64 * 1550, 128, 128, 64))
+    assert lib.sparse_attn_fused(big, a, a, a, 0.05, 0.9, a, a, a, 0, None, ws, 1 << 30, None) == 2
+    assert lib.sparse_attn_fused(sh, a, a, a, 0.0, 0.0, a, a, a, 0, None, ws, need, None) == 1   # k = p = 0
+    assert lib.sparse_attn_fused(sh, z, a, a, 0.05, 0.9, a, a, a, 0, None, ws, need, None) == 1
+    assert lib.sparse_attn_fused(sh, a, a, a, 0.05, 0.9, a, a, a, 3, None, ws, need, None) == 1
+    assert lib.sparse_attn_fused(sh, a, a, a, 0.05, 0.9, a, a, a, 0, None, ws, need - 1, None) == 1
+    assert lib.sparse_attn_fused(sh, a, a, a, 0.05, 0.9, a, a, a, 0, None, ctypes.c_void_p(16), need, None) == 1
+    assert lib.sparse_attn_fused(sh, a, a, a, 0.05, 0.9, a, a, a, 0, None, z, need, None) == 1

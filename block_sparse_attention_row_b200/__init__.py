@@ -11,7 +11,9 @@ from .capi import (EXPORTED, SparseAttnError, bwd_workspace_bytes, check_device_
                    sparse_attn_kmeans_permutation, sparse_attn_permute_rows,
                    permuted_sparse_attn, fused_workspace_bytes, sparse_attn_fused, version)
 
-__all__ = ["EXPORTED", "SparseAttnError", "bwd_workspace_bytes", "check_device_error", "sparse_attn_bwd", "host_workspace_bytes",
+from .sharding import head_range, head_shard
+
+__all__ = ["head_range", "head_shard", "EXPORTED", "SparseAttnError", "bwd_workspace_bytes", "check_device_error", "sparse_attn_bwd", "host_workspace_bytes",
            "load_library", "mask_workspace_bytes", "num_blocks", "sparse_attn", "sparse_attn_fwd",
            "sparse_attn_fwd_dense", "sparse_attn_host", "sparse_attn_mask", "sparse_attn_select",
            "sparse_attn_quantize_fp8", "sparse_attn_fwd_fp8", "sparse_attn_sparse_linear",

@@ -57,3 +57,72 @@ def test_weak_scaling_aggregation_two_gloo_ranks():
 def test_single_rank_aggregation_is_identity():
     import bench
     assert bench.aggregate_over_ranks(4.0, 7.0, 1, None) == (4.0, 7.0)
+
+
+def test_head_ranges_partition_the_heads():
+    from block_sparse_attention_row_b200 import head_range
+    for n in (0, 1, 5, 13, 40, 48, 97):
+        for world in (1, 2, 3, 4, 8):
+            got = [head_range(n, world, r) for r in range(world)]
+            assert got[0][0] == 0 and got[-1][1] == n
+            assert all(a[1] == b[0] for a, b in zip(got, got[1:]))          # contiguous, in rank order
+            sizes = [hi - lo for lo, hi in got]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        head_range(4, 2, 2)
+
+
+def _sharded_worker(rank, world, port, q):
+    import datetime
+    import sys
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import oracle as O
+    from block_sparse_attention_row_b200 import head_range, head_shard
+    from synth import make_qkv_custom
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    B, H, N, d, bq, bk, k, p = 2, 3, 300, 16, 64, 64, 0.2, 0.8
+    # Every rank holds the same layer (same seed) and takes its own heads of it.
+    Q, K, V = make_qkv_custom(B, H, N, d, seed=7, positional_field=True, sink_heads=(0,), uniform_heads=(1,))
+    Qs, Ks, Vs = (head_shard(x, world, rank) for x in (Q, K, V))
+    _, cnt, idx, _ = O.hybrid_mask(Qs, Ks, bq, bk, k, p)
+    Os, _ = O.block_sparse_attention(Qs, Ks, Vs, cnt, idx, bq, bk)
+    parts = [None] * world
+    dist.all_gather_object(parts, (head_range(B * H, world, rank), cnt, idx, Os))
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        _, cnt_w, idx_w, _ = O.hybrid_mask(Q, K, bq, bk, k, p)
+        O_w, _ = O.block_sparse_attention(Q, K, V, cnt_w, idx_w, bq, bk)
+        flat = lambda a: a.reshape((B * H,) + a.shape[2:])
+        ok = True
+        covered = []
+        for (lo, hi), c, i, o in parts:
+            covered += list(range(lo, hi))
+            ok &= np.array_equal(c[0], flat(cnt_w)[lo:hi]) and np.array_equal(i[0], flat(idx_w)[lo:hi])
+            ok &= np.array_equal(o[0], flat(O_w)[lo:hi])
+        q.put((ok, covered))
+    else:
+        q.put(None)
+
+
+def test_head_sharded_layer_equals_the_whole_layer_two_gloo_ranks():
+    """Two ranks each run the path (the oracle, on CPU) on their heads of one
+    layer; gathered, the shards equal the whole layer's lists and output."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ok, covered = next(r for r in res if r is not None)
+    assert covered == list(range(6))
+    assert ok

@@ -19,8 +19,9 @@
 // Kernels, per (batch, head):
 //   km_init_kernel     centroids = the tokens at floor(c N / C);
 //   km_assign_kernel   one thread per token, centroids staged in shared memory;
-//   km_sort_kernel     one warp per head: counting sort, stable by token order
-//                      (cluster offsets for the update, the permutation);
+//   km_sort_kernel     one CTA per head: counting sort over up to 8 warps
+//                      token ranges, stable by token order (cluster offsets
+//                      for the update, the permutation);
 //   km_update_kernel   one thread per (cluster, channel): sequential sums;
 //   permute_rows_kernel  Y[i] = X[perm[i]] or Y[perm[i]] = X[i].
 #pragma once
@@ -50,7 +51,7 @@ template <int D>
 __global__ void __launch_bounds__(AS_THREADS)
 km_assign_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ M, int32_t* __restrict__ ids,
                  int N, int C) {
-    __shared__ float ms[AS_CHUNK * D];
+    __shared__ __align__(16) float ms[AS_CHUNK * D];
     const int bh = blockIdx.y;
     const int t = blockIdx.x * AS_THREADS + threadIdx.x;
     const bool valid = t < N;
@@ -77,20 +78,33 @@ km_assign_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ 
     for (int c0 = 0; c0 < C; c0 += AS_CHUNK) {
         const int nc = min(AS_CHUNK, C - c0);
         __syncthreads();
-        for (int e = threadIdx.x; e < nc * D; e += AS_THREADS) ms[e] = Mh[(size_t)c0 * D + e];
+        // 16-byte loads, several in flight per thread (one L2 round trip per chunk).
+        const float4* src = reinterpret_cast<const float4*>(Mh + (size_t)c0 * D);
+        float4* dst = reinterpret_cast<float4*>(ms);
+#pragma unroll 8
+        for (int e = threadIdx.x; e < nc * (D / 4); e += AS_THREADS) dst[e] = __ldg(src + e);
         __syncthreads();
         int c = 0;
         for (; c + 4 <= nc; c += 4) {
-            const float* m0 = ms + c * D;
+            // Four centroids, their channels read 4 at a time (16-byte broadcast
+            // loads): the fp32 pipe, not instruction issue, bounds the loop.
+            const float4* m4 = reinterpret_cast<const float4*>(ms + c * D);
             float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
 #pragma unroll
-            for (int j = 0; j < D; ++j) {
-                const float a0 = __fsub_rn(x[j], m0[j]), a1 = __fsub_rn(x[j], m0[D + j]);
-                const float a2 = __fsub_rn(x[j], m0[2 * D + j]), a3 = __fsub_rn(x[j], m0[3 * D + j]);
-                d0 = __fadd_rn(d0, __fmul_rn(a0, a0));
-                d1 = __fadd_rn(d1, __fmul_rn(a1, a1));
-                d2 = __fadd_rn(d2, __fmul_rn(a2, a2));
-                d3 = __fadd_rn(d3, __fmul_rn(a3, a3));
+            for (int j4 = 0; j4 < D / 4; ++j4) {
+                const float4 q0 = m4[j4], q1 = m4[D / 4 + j4], q2 = m4[2 * (D / 4) + j4], q3 = m4[3 * (D / 4) + j4];
+                const float c0[4] = {q0.x, q0.y, q0.z, q0.w}, c1[4] = {q1.x, q1.y, q1.z, q1.w};
+                const float c2[4] = {q2.x, q2.y, q2.z, q2.w}, c3[4] = {q3.x, q3.y, q3.z, q3.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * j4 + e;
+                    const float a0 = __fsub_rn(x[j], c0[e]), a1 = __fsub_rn(x[j], c1[e]);
+                    const float a2 = __fsub_rn(x[j], c2[e]), a3 = __fsub_rn(x[j], c3[e]);
+                    d0 = __fadd_rn(d0, __fmul_rn(a0, a0));
+                    d1 = __fadd_rn(d1, __fmul_rn(a1, a1));
+                    d2 = __fadd_rn(d2, __fmul_rn(a2, a2));
+                    d3 = __fadd_rn(d3, __fmul_rn(a3, a3));
+                }
             }
             if (d0 < best) { best = d0; best_c = c0 + c; }
             if (d1 < best) { best = d1; best_c = c0 + c + 1; }
@@ -111,44 +125,71 @@ km_assign_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ 
     if (valid) ids[(size_t)bh * N + t] = best_c;
 }
 
-// One warp per head: histogram of the cluster ids (shared memory), exclusive
-// scan into offsets, then the tokens are placed in ascending order, 32 at a
-// time: lanes with the same id (match) take consecutive positions in lane
-// order, and their group's leader advances the cluster's cursor. off gets the
-// C + 1 cluster offsets (off[C] = N).
-__global__ void __launch_bounds__(32)
+// One CTA per head, W = blockDim.x / 32 warps, warp w taking the w-th
+// contiguous range of the tokens: per-warp histograms of the cluster ids
+// (shared memory), an exclusive scan of the totals into the cluster offsets,
+// per-warp cursors (a cluster's offset plus the counts of the warps before),
+// then each warp places its tokens in ascending order, 32 at a time: lanes
+// with the same id (match) take consecutive positions in lane order and
+// their group's leader advances the cursor. The order within a cluster is
+// therefore the token order. off gets the C + 1 cluster offsets (off[C] = N).
+// Shared memory: (W + 1) * C ints.
+__global__ void __launch_bounds__(256)
 km_sort_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ perm, int32_t* __restrict__ off, int N, int C) {
-    extern __shared__ int32_t cur[];   // [C]
-    const int bh = blockIdx.x, lane = threadIdx.x;
+    extern __shared__ int32_t sort_smem[];
+    const int W = blockDim.x / 32;
+    const int bh = blockIdx.x, warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    int32_t* tot = sort_smem;                    // [C]: totals, then cluster offsets
+    int32_t* cur = sort_smem + C + warp * C;     // [C]: this warp's counts, then cursors
     const int32_t* id = ids + (size_t)bh * N;
     int32_t* pm = perm + (size_t)bh * N;
     int32_t* of = off + (size_t)bh * (C + 1);
-    for (int c = lane; c < C; c += 32) cur[c] = 0;
-    __syncwarp();
-    for (int t = lane; t < N; t += 32) atomicAdd(&cur[id[t]], 1);
-    __syncwarp();
-    int run = 0;   // exclusive scan, 32 clusters at a time
-    for (int c0 = 0; c0 < C; c0 += 32) {
-        const int c = c0 + lane;
-        const int v = c < C ? cur[c] : 0;
-        int incl = v;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        if (c < C) {
-            cur[c] = run + incl - v;
-            of[c] = run + incl - v;
-        }
-        run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    const int span = (N + W - 1) / W;
+    const int t_lo = min(N, warp * span), t_hi = min(N, t_lo + span);
+    for (int e = threadIdx.x; e < (W + 1) * C; e += blockDim.x) sort_smem[e] = 0;
+    __syncthreads();
+    for (int t = t_lo + lane; t < t_hi; t += 32) atomicAdd(&cur[id[t]], 1);
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int s = 0;
+        for (int w = 0; w < W; ++w) s += sort_smem[C + w * C + c];
+        tot[c] = s;
     }
-    if (lane == 0) of[C] = run;
-    __syncwarp();
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;   // exclusive scan, 32 clusters at a time
+        for (int c0 = 0; c0 < C; c0 += 32) {
+            const int c = c0 + lane;
+            const int v = c < C ? tot[c] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (c < C) {
+                tot[c] = run + incl - v;
+                of[c] = run + incl - v;
+            }
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) of[C] = run;
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        int run = tot[c];
+        for (int w = 0; w < W; ++w) {
+            int32_t* h = sort_smem + C + w * C + c;
+            const int n = *h;
+            *h = run;
+            run += n;
+        }
+    }
+    __syncthreads();
     const uint32_t lt = (1u << lane) - 1u;
-    for (int base = 0; base < N; base += 32) {
+    for (int base = t_lo; base < t_hi; base += 32) {
         const int t = base + lane;
-        const bool valid = t < N;
+        const bool valid = t < t_hi;
         const int c = valid ? id[t] : -1 - lane;   // invalid lanes match nobody
         const uint32_t grp = __match_any_sync(0xFFFFFFFFu, c);
         if (valid) pm[cur[c] + __popc(grp & lt)] = t;
@@ -156,6 +197,13 @@ km_sort_kernel(const int32_t* __restrict__ ids, int32_t* __restrict__ perm, int3
         if (valid && (grp & lt) == 0) cur[c] += __popc(grp);
         __syncwarp();
     }
+}
+
+// Warps of km_sort_kernel for C clusters: as many as (W + 1) * C ints of
+// shared memory allow within `budget` bytes, at most 8.
+inline int km_sort_warps(int C, size_t budget) {
+    long long w = (long long)(budget / (4 * (size_t)C)) - 1;
+    return (int)(w < 1 ? 1 : (w > 8 ? 8 : w));
 }
 
 // One CTA per (cluster, head), one thread per channel: the members are

@@ -602,10 +602,17 @@ sa_status launch_kmeans(const Dims& g, const void* X, int C, int iters, const fl
         if ((s = cuda_check(cudaGetLastError(), "km_init_kernel launch")) != SA_OK) return s;
     }
     const dim3 ag((g.N + sa::km::AS_THREADS - 1) / sa::km::AS_THREADS, g.BH);
+    constexpr size_t SORT_SMEM_BUDGET = 200 * 1024;
+    const int sw = sa::km::km_sort_warps(C, SORT_SMEM_BUDGET);
+    const size_t sort_smem = (size_t)(sw + 1) * C * sizeof(int32_t);
+    if ((s = cuda_check(cudaFuncSetAttribute(sa::km::km_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SORT_SMEM_BUDGET),
+                        "km_sort_kernel shared-memory attribute")) != SA_OK)
+        return s;
     for (int it = 0; it <= iters; ++it) {
         sa::km::km_assign_kernel<D><<<ag, sa::km::AS_THREADS, 0, st>>>(x, M, ids, g.N, C);
         if ((s = cuda_check(cudaGetLastError(), "km_assign_kernel launch")) != SA_OK) return s;
-        sa::km::km_sort_kernel<<<g.BH, 32, (size_t)C * sizeof(int32_t), st>>>(ids, perm, off, g.N, C);
+        sa::km::km_sort_kernel<<<g.BH, 32 * sw, sort_smem, st>>>(ids, perm, off, g.N, C);
         if ((s = cuda_check(cudaGetLastError(), "km_sort_kernel launch")) != SA_OK) return s;
         if (it == iters) break;   // the final assignment is not followed by an update
         sa::km::km_update_kernel<D><<<dim3(C, g.BH), D, 0, st>>>(x, perm, off, M, g.N, C);

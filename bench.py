@@ -38,6 +38,7 @@ PERM_C = 256
 PERM_COLD_ITERS = 8
 PERM_WARM_ITERS = 2
 FWD_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_attn_kernel.cuh",
+               "block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
                "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]
 MASK_SOURCES = ["block_sparse_attention_row_b200/csrc/sa_mask_kernels.cuh",
                 "block_sparse_attention_row_b200/csrc/sa_ptx.cuh"]

@@ -85,6 +85,12 @@ def random_rows(seed, n_rows, n, kind):
         L = rng.integers(0, 4, size=(n_rows, n)).astype(np.float64)
         P = 2.0 ** (L - 8)
         P /= P.sum(1, keepdims=True)
+    elif kind == "all_equal":  # one value repeated: every boundary is a tie
+        return np.full((n_rows, n), np.float32(1.0 / n), dtype=np.float32)
+    elif kind == "low_bits":  # fp32 values that differ only in their last few mantissa bits
+        base = np.float32(1.0 / n)
+        steps = rng.integers(0, 16, size=(n_rows, n)).astype(np.uint32)
+        return (np.full((n_rows, n), base, dtype=np.float32).view(np.uint32) - steps).view(np.float32)   # <= 1/n
     else:
         raise ValueError(kind)
     return P.astype(np.float32)

@@ -86,7 +86,8 @@ def test_select_hand_rows():
             assert idx[0, 0, i, :cnt[0, 0, i]].tolist() == r["kept"], r["name"]
 
 
-@pytest.mark.parametrize("kind", ["dirichlet_flat", "dirichlet_peaky", "softmax_logits", "quantised_ties"])
+@pytest.mark.parametrize("kind", ["dirichlet_flat", "dirichlet_peaky", "softmax_logits", "quantised_ties", "all_equal",
+                                  "low_bits"])
 @pytest.mark.parametrize("n_k", [1, 7, 64, 275, 1182, 4096])
 def test_select_random_rows_bit_exact(kind, n_k):
     from _pins import random_rows

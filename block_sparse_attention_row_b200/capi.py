@@ -477,11 +477,13 @@ def kmeans_workspace_bytes(B, H, N, d, C, bq: int = 64, bk: int = 64) -> int:
 
 
 def sparse_attn_kmeans_permutation(X: torch.Tensor, C: int, iters: int, *, init: Optional[torch.Tensor] = None,
+                                   out_centroids: Optional[torch.Tensor] = None,
                                    workspace: Optional[torch.Tensor] = None, stream=None):
     """k-means of every head's token vectors (Sparse VideoGen2 §2A) and the
     stable permutation by cluster. X bf16 [B, H, N, d]; init fp32
-    [B, H, C, d] (cached centroids) or None. Returns (ids int32 [B, H, N],
-    perm int32 [B, H, N], centroids fp32 [B, H, C, d])."""
+    [B, H, C, d] (cached centroids) or None; out_centroids: where the final
+    centroids go (may be init itself: the cache updated in place). Returns
+    (ids int32 [B, H, N], perm int32 [B, H, N], centroids fp32 [B, H, C, d])."""
     if not isinstance(X, torch.Tensor) or not X.is_cuda or X.dtype != torch.bfloat16 or X.dim() != 4 \
             or not X.is_contiguous():
         raise ValueError("X must be a contiguous bf16 CUDA tensor [B, H, N, d]")
@@ -499,7 +501,12 @@ def sparse_attn_kmeans_permutation(X: torch.Tensor, C: int, iters: int, *, init:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     ids = torch.empty((B, H, N), dtype=torch.int32, device=dev)
     perm = torch.empty((B, H, N), dtype=torch.int32, device=dev)
-    M = torch.empty((B, H, int(C), d), dtype=torch.float32, device=dev)
+    if out_centroids is None:
+        M = torch.empty((B, H, int(C), d), dtype=torch.float32, device=dev)
+    else:
+        M = out_centroids
+        if M.dtype != torch.float32 or tuple(M.shape) != (B, H, int(C), d) or not M.is_contiguous() or M.device != dev:
+            raise ValueError(f"out_centroids must be a contiguous fp32 tensor {(B, H, int(C), d)} on {dev}")
     st = lib.sparse_attn_kmeans_permutation(ctypes.byref(shape), _ptr(X), int(C), int(iters), _ptr(init),
                                             _ptr(ids), _ptr(perm), _ptr(M), _ptr(workspace),
                                             workspace.numel() * workspace.element_size(), _stream(dev, stream))

@@ -594,7 +594,9 @@ sa_status launch_kmeans(const Dims& g, const void* X, int C, int iters, const fl
     auto* x = reinterpret_cast<const __nv_bfloat16*>(X);
     sa_status s;
     if (init) {
-        if ((s = cuda_check(cudaMemcpyAsync(M, init, (size_t)g.BH * C * D * sizeof(float), cudaMemcpyDeviceToDevice, st),
+        // Cached centroids (the output buffer itself when the caller updates them in place).
+        if (init != M &&
+            (s = cuda_check(cudaMemcpyAsync(M, init, (size_t)g.BH * C * D * sizeof(float), cudaMemcpyDeviceToDevice, st),
                             "copy the initial centroids")) != SA_OK)
             return s;
     } else {

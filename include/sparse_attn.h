@@ -251,7 +251,8 @@ size_t sparse_attn_kmeans_workspace_bytes(const sa_shape* shape, int C);
  *          min(N, 8192); iters in [0, 100]; init_or_null fp32 [B,H,C,d].
  * Outputs: ids int32 [B,H,N] (final cluster of every token), perm int32
  *          [B,H,N], centroids fp32 [B,H,C,d] (after `iters` updates; may be
- *          the same buffer as init_or_null).
+ *          the same buffer as init_or_null, which is then updated in place;
+ *          any other overlap of the two is not allowed).
  * workspace: device, sparse_attn_kmeans_workspace_bytes(shape, C) bytes,
  *          256-byte aligned; workspace_bytes is checked against that size.
  * Device pointers 16-byte aligned. Errors: SA_ERR_INVALID_ARG on a bad

@@ -68,9 +68,11 @@ def test_kmeans_from_cached_centroids():
     ids, perm, M = sparse_attn_kmeans_permutation(Q, 50, 3, init=M0)
     check_device_error(Q.device)
     _assert_exact(ids, perm, M, _oracle_heads(Qh, 50, 3, heads, init=init_h), heads)
-    # The same buffer may serve as init and as output.
-    ids2, perm2, M2 = sparse_attn_kmeans_permutation(Q, 50, 3, init=M0.clone())
-    assert torch.equal(ids2, ids) and torch.equal(perm2, perm) and torch.equal(M2, M)
+    # The same buffer may serve as init and as output (the cache updated in place).
+    cache = M0.clone()
+    ids2, perm2, M2 = sparse_attn_kmeans_permutation(Q, 50, 3, init=cache, out_centroids=cache)
+    assert M2.data_ptr() == cache.data_ptr()
+    assert torch.equal(ids2, ids) and torch.equal(perm2, perm) and torch.equal(cache, M)
 
 
 @pytest.mark.parametrize("N,d,C,iters", [(1000, 64, 1, 3), (200, 128, 200, 2), (777, 64, 33, 0),

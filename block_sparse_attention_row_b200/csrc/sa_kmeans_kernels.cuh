@@ -225,26 +225,37 @@ km_update_kernel(const __nv_bfloat16* __restrict__ X, const int32_t* __restrict_
 }
 
 // Rows of [BH, N, D] elements of ESIZE bytes (2: bf16, 4: fp32): inverse = 0
-// gathers Y[i] = X[perm[i]], inverse = 1 scatters Y[perm[i]] = X[i]. One warp
-// per row, 16-byte copies. An entry outside [0, N) is recorded as a device
+// gathers Y[i] = X[perm[i]], inverse = 1 scatters Y[perm[i]] = X[i]. Each
+// row is ROW_BYTES / 16 lanes, one 16-byte chunk each (a warp moves 1, 2 or
+// 4 rows at once). An entry outside [0, N) is recorded as a device
 // assertion and its row is skipped.
+template <int ROW_BYTES>
+struct PermuteShape {
+    static constexpr int LANES = ROW_BYTES / 16;          // lanes per row
+    static constexpr int ROWS_PER_WARP = 32 / LANES;
+    static constexpr int ROWS_PER_CTA = 8 * ROWS_PER_WARP;   // 256 threads
+    static_assert(LANES >= 1 && LANES <= 32 && 32 % LANES == 0, "row of 16..512 bytes");
+};
+
 template <int ROW_BYTES>
 __global__ void __launch_bounds__(256)
 permute_rows_kernel(const uint8_t* __restrict__ X, const int32_t* __restrict__ perm, uint8_t* __restrict__ Y, int N,
                     int inverse) {
+    using S = PermuteShape<ROW_BYTES>;
     const int bh = blockIdx.y;
-    const int i = blockIdx.x * 8 + threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int i = blockIdx.x * S::ROWS_PER_CTA + warp * S::ROWS_PER_WARP + lane / S::LANES;
+    const int c = lane % S::LANES;
     if (i >= N) return;
     const int p = perm[(size_t)bh * N + i];
     if (p < 0 || p >= N) {                    // not a permutation entry: reported, row skipped
-        if (lane == 0) record_error(SA_STATUS_DEVICE_ASSERT, 0x9E00u);
+        if (c == 0) record_error(SA_STATUS_DEVICE_ASSERT, 0x9E00u);
         return;
     }
     const int src = inverse ? i : p, dst = inverse ? p : i;
     const uint4* s = reinterpret_cast<const uint4*>(X + ((size_t)bh * N + src) * ROW_BYTES);
     uint4* d = reinterpret_cast<uint4*>(Y + ((size_t)bh * N + dst) * ROW_BYTES);
-    for (int e = lane; e < ROW_BYTES / 16; e += 32) d[e] = __ldg(s + e);
+    d[c] = __ldg(s + c);
 }
 
 }  // namespace km

@@ -706,13 +706,17 @@ sa_status sparse_attn_permute_rows(const sa_shape* shape, const void* X, const i
     if (!aligned16(X) || !aligned16(perm) || !aligned16(Y))
         return fail(SA_ERR_INVALID_ARG, "misaligned pointer (16 bytes required)");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const dim3 grid((g.N + 7) / 8, g.BH);
     auto* x = reinterpret_cast<const uint8_t*>(X);
     auto* y = reinterpret_cast<uint8_t*>(Y);
     const int row_bytes = g.d * (dtype == SA_F32 ? 4 : 2);
-    if (row_bytes == 128) sa::km::permute_rows_kernel<128><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
-    else if (row_bytes == 256) sa::km::permute_rows_kernel<256><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
-    else sa::km::permute_rows_kernel<512><<<grid, 256, 0, st>>>(x, perm, y, g.N, inverse ? 1 : 0);
+    auto grid = [&](int rows_per_cta) { return dim3((g.N + rows_per_cta - 1) / rows_per_cta, g.BH); };
+    const int inv = inverse ? 1 : 0;
+    if (row_bytes == 128)
+        sa::km::permute_rows_kernel<128><<<grid(sa::km::PermuteShape<128>::ROWS_PER_CTA), 256, 0, st>>>(x, perm, y, g.N, inv);
+    else if (row_bytes == 256)
+        sa::km::permute_rows_kernel<256><<<grid(sa::km::PermuteShape<256>::ROWS_PER_CTA), 256, 0, st>>>(x, perm, y, g.N, inv);
+    else
+        sa::km::permute_rows_kernel<512><<<grid(sa::km::PermuteShape<512>::ROWS_PER_CTA), 256, 0, st>>>(x, perm, y, g.N, inv);
     if ((s = cuda_check(cudaGetLastError(), "permute_rows_kernel launch")) != SA_OK) return s;
     return ok();
 }

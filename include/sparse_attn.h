@@ -17,6 +17,22 @@
  * compressed score from pooled Q and K) and "Sparse VideoGen2" §1 (mean
  * pooling of contiguous token blocks).
  *
+ * Entry points (each documented at its declaration below)
+ * ---------------------------------------------------------
+ *   sparse_attn_mask[_noalloc]       steps 1-3: pooled scores, hybrid lists
+ *   sparse_attn_select               step 3 alone, on given scores
+ *   sparse_attn_fwd[_dense]          step 4 over the lists (or every block)
+ *   sparse_attn_fused                steps 1-4 in one cooperative launch
+ *   sparse_attn_quantize_fp8,
+ *   sparse_attn_fwd_fp8              step 4 with e4m3 Q and K (per-block scales)
+ *   sparse_attn_sparse_linear        SLA2's alpha mix with a linear branch
+ *   sparse_attn_kmeans_permutation,
+ *   sparse_attn_permute_rows         Sparse VideoGen2's semantic permutation
+ *   sparse_attn_bwd                  gradients of step 4, lists held fixed
+ *   sparse_attn_host                 steps 1-4 on host buffers, pipelined
+ *   *_workspace_bytes, sparse_attn_check_device_error, sparse_attn_last_error,
+ *   sparse_attn_version
+ *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Tensors are dense, row-major, with no padding:

@@ -126,3 +126,19 @@ def test_head_sharded_layer_equals_the_whole_layer_two_gloo_ranks():
     ok, covered = next(r for r in res if r is not None)
     assert covered == list(range(6))
     assert ok
+
+
+def test_head_shard_is_a_contiguous_view_of_the_layer():
+    import torch
+    from block_sparse_attention_row_b200 import head_range, head_shard
+    X = torch.arange(2 * 5 * 3 * 4, dtype=torch.float32).reshape(2, 5, 3, 4)
+    flat = X.reshape(10, 3, 4)
+    for world in (1, 3, 4):
+        for r in range(world):
+            lo, hi = head_range(10, world, r)
+            S = head_shard(X, world, r)
+            assert S.shape == (1, hi - lo, 3, 4) and S.is_contiguous()
+            assert S.data_ptr() == flat[lo:].data_ptr() if hi > lo else True
+            assert torch.equal(S[0], flat[lo:hi])
+    with pytest.raises(ValueError):
+        head_shard(X.transpose(1, 2), 2, 0)
